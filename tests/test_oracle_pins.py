@@ -1,0 +1,287 @@
+"""Pins for the CPU oracle, against facts that come from outside the oracle.
+
+Every check compares the oracle with something it does not share code with:
+brute-force sums written as loops, closed forms, special cases that reduce
+to plain attention, brute force over subsets, and the worked example printed
+on "XAttention 计算步骤详解及示例" (§2). A few tests plant a plausible mistake
+in a copy of the oracle and check that a pin catches it.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle.xattn_oracle as O
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(1234)
+
+
+def _rand(*shape, scale=1.0):
+    return rng.standard_normal(shape) * scale
+
+
+# ---------------------------------------------------------------- P1 --------
+@pytest.mark.parametrize("S", [1, 2, 4, 8])
+def test_reshape_equals_bruteforce_antidiagonal(S):
+    """Alg. 1's reshaped product equals the antidiagonal sum of every S x S
+    tile of Q K^T (§2.1: lower-left to upper-right)."""
+    q, k = _rand(32, 4), _rand(32, 4)
+    got = O.reshaped_logits(q, k, S)
+    want = O.antidiagonal_sums_bruteforce(q, k, S)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_main_diagonal_mistake_is_caught():
+    """Planted mistake: stacking query slices in increasing order gives the
+    main diagonal, which the brute-force pin rejects."""
+    q, k = _rand(32, 4), _rand(32, 4)
+    S = 4
+    wrong = np.concatenate([q[i::S] for i in range(S)], axis=1) @ O.reshape_keys(k, S).T
+    want = O.antidiagonal_sums_bruteforce(q, k, S)
+    assert np.max(np.abs(wrong - want)) > 1e-3
+
+
+# ---------------------------------------------------------------- scale -----
+def _group_constant(nt, d, S, scale=1.0):
+    base = _rand(nt, d, scale=scale)
+    return base, np.repeat(base, S, axis=0)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_scale_sqrt_dS_closed_form(causal):
+    """Queries and keys constant within each S-group turn A_approx into plain
+    attention of (sqrt(S) q_hat, k_hat). So the scale 1/sqrt(d_h S) is pinned
+    against the independent naive attention routine."""
+    S, d, B = 4, 8, 16
+    r = B // S
+    qh, q = _group_constant(16, d, S, 0.7)
+    kh, k = _group_constant(16, d, S, 0.7)
+    P = O.block_probs_head(q, k, B, S, causal)
+    _, probs = O.dense_attention_naive(math.sqrt(S) * qh, kh, np.zeros((16, 1)), causal)
+    NB = q.shape[0] // B
+    want = probs.reshape(NB, r, NB, r).sum(axis=(1, 3)) / r
+    np.testing.assert_allclose(P, want, rtol=0, atol=1e-12)
+
+
+def test_wrong_scale_is_caught():
+    """Planted mistake: scaling by 1/sqrt(d) alone changes P beyond 1e-6."""
+    S, d, B = 4, 8, 16
+    qh, q = _group_constant(16, d, S, 0.7)
+    kh, k = _group_constant(16, d, S, 0.7)
+    good = O.block_probs_head(q, k, B, S, True)
+    bad = O.block_probs_head(q * math.sqrt(S), k, B, S, True)
+    assert np.max(np.abs(good - bad)) > 1e-6
+
+
+# ---------------------------------------------------------------- P2 --------
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("S", [2, 4, 8])
+def test_rows_are_distributions(causal, S):
+    """Each softmax row sums to 1, so each P row sums to 1 (tau in (0, 1]).
+    Causal rows are 0 above the diagonal."""
+    q, k = _rand(256, 16), _rand(256, 16)
+    P = O.block_probs_head(q, k, 32, S, causal)
+    np.testing.assert_allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    assert (P >= 0).all()
+    if causal:
+        assert np.all(P[np.triu_indices(P.shape[0], 1)] == 0.0)
+    x = O.reshaped_logits(q, k, S) / math.sqrt(16 * S)
+    A = O.approx_attention_rows(x, 0, causal)
+    np.testing.assert_allclose(A.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    if causal:
+        assert A[0, 0] == 1.0   # reshaped row 0 sees only reshaped column 0
+
+
+# ---------------------------------------------------------------- P3 --------
+@pytest.mark.parametrize("causal", [True, False])
+def test_stride_one_is_exact_attention(causal):
+    """With S = 1 the reshape is the identity and A_approx is exact attention,
+    so P is the block mean of the naive attention probabilities."""
+    q, k = _rand(48, 4), _rand(48, 4)
+    B = 8
+    P = O.block_probs_head(q, k, B, 1, causal)
+    _, probs = O.dense_attention_naive(q, k, np.zeros((48, 1)), causal)
+    NB = 48 // B
+    want = probs.reshape(NB, B, NB, B).sum(axis=(1, 3)) / B
+    np.testing.assert_allclose(P, want, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- P4 --------
+@pytest.mark.parametrize("causal", [True, False])
+def test_tau_one_selects_everything_allowed(causal):
+    q, k = _rand(256, 8), _rand(256, 8)
+    P = O.block_probs_head(q, k, 32, 4, causal)[None, None]
+    mask, lists = O.select_blocks(P, [1.0], causal)
+    NB = P.shape[-1]
+    want = np.tril(np.ones((NB, NB), bool)) if causal else np.ones((NB, NB), bool)
+    assert (mask[0, 0] == want).all()
+
+
+# ---------------------------------------------------------------- P5 --------
+@pytest.mark.parametrize("causal", [True, False])
+def test_dense_mask_sparse_attention_is_naive_attention(causal):
+    q, k, v = _rand(32, 4), _rand(32, 4), _rand(32, 3)
+    B = 8
+    NB = 4
+    lists = {b: list(range(b + 1 if causal else NB)) for b in range(NB)}
+    Os, lse = O.sparse_attention_head(q, k, v, B, causal, lists)
+    On, _ = O.dense_attention_naive(q, k, v, causal)
+    np.testing.assert_allclose(Os, On, rtol=0, atol=1e-12)
+    raw = O.dense_scores(q, k) / math.sqrt(4)
+    for i in range(32):
+        n = i + 1 if causal else 32
+        want = math.log(math.fsum(math.exp(x) for x in raw[i, :n]))
+        assert abs(lse[i] - want) < 1e-12
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_sparse_lists_match_filtered_naive_attention(causal):
+    """Any block list equals naive attention with the unlisted blocks
+    filtered out (block 0 is in every list, so no row is empty)."""
+    q, k, v = _rand(64, 4), _rand(64, 4), _rand(64, 5)
+    B, NB = 8, 8
+    lists = {}
+    for b in range(NB):
+        n = b + 1 if causal else NB
+        pick = {0} | {j for j in range(n) if rng.random() < 0.5}
+        lists[b] = sorted(pick)
+    Os, _ = O.sparse_attention_head(q, k, v, B, causal, lists)
+    On, _ = O.dense_attention_naive(q, k, v, causal,
+                                    allowed=lambda i, j: (j // B) in lists[i // B])
+    np.testing.assert_allclose(Os, On, rtol=0, atol=1e-12)
+
+
+def test_empty_list_gives_zero_row():
+    q, k, v = _rand(16, 4), _rand(16, 4), _rand(16, 2)
+    Os, lse = O.sparse_attention_head(q, k, v, 8, True, {0: [0], 1: []})
+    assert np.all(Os[8:] == 0.0) and np.all(np.isneginf(lse[8:]))
+
+
+# ---------------------------------------------------------------- P6 --------
+def _brute_minimal(p, tau):
+    n = len(p)
+    for size in range(1, n + 1):
+        best = None
+        for sub in itertools.combinations(range(n), size):
+            s = math.fsum(p[i] for i in sub)
+            if s >= tau:
+                key = (-s, sub)
+                if best is None or key < best:
+                    best = key
+        if best is not None:
+            return list(best[1])
+    return list(range(n))
+
+
+@pytest.mark.parametrize("trial", range(40))
+def test_find_blocks_minimal_and_tie_break(trial):
+    """Brute force over all subsets: the chosen set has the smallest size that
+    reaches tau. Among the sets of that size with the largest sum it is the
+    one with the lowest indices (ties go to the lower block index)."""
+    n = int(rng.integers(1, 11))
+    p = rng.dirichlet(np.ones(n) * 0.5)
+    if trial % 3 == 0:           # plant exact ties
+        p = np.round(p * 8) / 8
+        p = p / p.sum() if p.sum() > 0 else np.full(n, 1.0 / n)
+    cs = np.cumsum(np.sort(p)[::-1])
+    while True:
+        tau = float(rng.uniform(0.05, 0.999))
+        if np.min(np.abs(cs - tau)) > 1e-9:
+            break
+    got = list(O.find_blocks(p, tau))
+    want = sorted(_brute_minimal(list(p), tau))
+    assert got == want
+    order = np.lexsort((np.arange(n), -p))
+    csum = np.cumsum(p[order])
+    k = len(got)
+    if csum[-1] >= tau:
+        assert csum[k - 1] >= tau and (k == 1 or csum[k - 2] < tau)
+
+
+def test_find_blocks_unreached_takes_all():
+    assert list(O.find_blocks(np.array([0.3, 0.3]), 0.9)) == [0, 1]
+
+
+# ---------------------------------------------------------------- P7 --------
+def test_worked_example_selection():
+    with open(os.path.join(GOLD, "find_blocks_worked_example.json")) as f:
+        g = json.load(f)
+    assert list(O.find_blocks(np.array(g["p"]), g["tau"])) == g["selected"]
+
+
+def test_worked_example_raw_scores():
+    with open(os.path.join(GOLD, "raw_scores_worked_example.json")) as f:
+        g = json.load(f)
+    q, k = np.array(g["Q"]), np.array(g["K"])
+    assert (O.dense_scores(q, k) == np.array(g["QKt"])).all()
+    assert (O.reshaped_logits(q, np.vstack([k, k[:1]])[:3], 1) == np.array(g["QKt"])).all()
+
+
+# ---------------------------------------------------------------- P8 --------
+def test_vertical_line_is_detected():
+    """§2.1: every key meets the antidiagonal of every tile in its column. A
+    single dominant key k* makes every later block row put almost all its mass
+    on k*'s block, and tau = 0.9 keeps only that block."""
+    L, d, B, S = 256, 32, 32, 4
+    q, k = _rand(L, d, scale=0.1), _rand(L, d, scale=0.1)
+    u = _rand(d)
+    u /= np.linalg.norm(u)
+    kstar = 77
+    q += u
+    k[kstar] += 400.0 * u
+    P = O.block_probs_head(q, k, B, S, True)
+    jb = kstar // B
+    r = B // S
+    first_full = -(-(kstar // S) // r)      # first block whose rows all see k*
+    for b in range(max(first_full, jb + 1), L // B):
+        assert P[b, jb] >= 0.99
+        assert list(O.find_blocks(P[b, : b + 1], 0.9)) == [jb]
+
+
+# ---------------------------------------------------------------- P9 --------
+@pytest.mark.parametrize("delta,seen", [(2, False), (4, False), (3, True), (1, True)])
+def test_antidiagonal_parity_orientation(delta, seen):
+    """For even S, antidiagonal cells have q - k odd. A slash at an even
+    offset is invisible, one at an odd offset is seen. A main-diagonal scorer
+    (the wrong orientation) shows the opposite parity, so this pins it."""
+    L, S = 32, 4
+    q = np.eye(L)
+    k = np.zeros((L, L))
+    for j in range(L - delta):
+        k[j, j + delta] = 1.0           # q_i . k_j = 1 iff i - j = delta
+    x = O.reshaped_logits(q, k, S)
+    assert (np.abs(x).sum() > 0) == seen
+    for t in range(L // S):
+        for c in range(L // S):
+            want = sum(1 for i in range(S) if t * S + S - 1 - i == c * S + i + delta)
+            assert x[t, c] == want
+    main = np.concatenate([q[i::S] for i in range(S)], axis=1) @ O.reshape_keys(k, S).T
+    assert (np.abs(main).sum() > 0) == (delta % S == 0)
+
+
+# ---------------------------------------------------------------- GQA -------
+def test_gqa_head_mapping():
+    """Query head h reads KV head h // (Hq / Hkv), not h % Hkv."""
+    hq, hkv, L, d = 4, 2, 64, 8
+    Q = _rand(1, hq, L, d)
+    K = _rand(1, hkv, L, d)
+    K[0, 1] *= 3.0
+    P = O.block_probs(Q, K, 16, 4, True)
+    for h in range(hq):
+        want = O.block_probs_head(Q[0, h], K[0, h // 2], 16, 4, True)
+        np.testing.assert_allclose(P[0, h], want, rtol=0, atol=0)
+    wrong = O.block_probs_head(Q[0, 1], K[0, 1], 16, 4, True)
+    assert np.max(np.abs(wrong - P[0, 1])) > 1e-6
+
+
+def test_q_block_subset_equals_full():
+    """Filling only some query blocks gives the same rows as the full run."""
+    q, k = _rand(512, 8), _rand(512, 8)
+    full = O.block_probs_head(q, k, 64, 8, True, chunk_rows=16)
+    part = O.block_probs_head(q, k, 64, 8, True, q_blocks=[0, 3, 7])
+    for b in (0, 3, 7):
+        np.testing.assert_allclose(part[b], full[b], rtol=0, atol=1e-14)
