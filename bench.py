@@ -1,0 +1,368 @@
+#!/usr/bin/env python3
+"""Benchmark of the XAttention prefill attention step (score + select + sparse).
+
+One step = one layer's prefill attention on the 128K Llama-3.1-8B-shaped
+workload (32 query / 8 KV heads, d = 128, L = 131072, bf16, causal, B = 128,
+S = 16, per-head tau from {0.8, 0.85, 0.9, 0.95}): xattn_score, xattn_select
+and xattn_sparse_attn through the C ABI, inputs resident in HBM.
+
+Prints one JSON line (rank 0). Multi-GPU runs (torchrun) are independent
+replicas: every rank runs the same layer, with no collective in the data path;
+the timed region is bracketed by a barrier and the max over ranks is reported.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill attn ms/layer at 128K (score+select+sparse); dense-equiv TFLOP/s, %peak"
+WORKLOAD = "c2"
+
+
+def peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=d["hbm_gbs"], bf16=d["bf16_tflops"],
+                    bf16_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def workload_config(prob) -> dict:
+    return {
+        "workload": f"llama3.1-8b attention layer, L={prob.L}, hq={prob.hq}/hkv={prob.hkv}, "
+                    f"d={prob.d}, bf16, causal, B={prob.B}, S={prob.S}, "
+                    "tau per head from {0.8,0.85,0.9,0.95}",
+        "L": prob.L, "hq": prob.hq, "hkv": prob.hkv, "d": prob.d, "B": prob.B, "S": prob.S,
+        "causal": prob.causal, "global_batch": prob.batch,
+        "l2": "no flush: inputs (Q/K/V 1.5 GB) and scoring partials (0.54 GB) exceed the 126 MB L2",
+        "parallelism": "replicas",
+    }
+
+
+def dense_equiv_flops(prob) -> float:
+    L = prob.L
+    pairs = L * (L + 1) / 2 if prob.causal else L * L
+    return 4.0 * prob.d * prob.hq * prob.batch * pairs
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        load = [s for s in sm if s > 0]
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_sample(prob, n_blocks: int = 48) -> dict:
+    """Times the fp64 oracle on one query head and an evenly spread sample of
+    query blocks (score, select, attention), scaled to the whole layer."""
+    import oracle.xattn_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        cores = os.cpu_count() or 1
+    NB = prob.NB
+    h = 0
+    step = max(1, NB // n_blocks)
+    blocks = list(range(step - 1, NB, step))[:n_blocks]
+    t0 = time.perf_counter()
+    P = O.block_probs(prob.Q, prob.K, prob.B, prob.S, prob.causal, heads=[h], q_blocks=blocks)
+    _, lists = O.select_blocks(P, prob.tau, prob.causal, heads=[h], q_blocks=blocks)
+    O.sparse_attention(prob.Q, prob.K, prob.V, prob.B, prob.causal, lists, heads=[h],
+                       q_blocks=blocks)
+    dt = time.perf_counter() - t0
+    units_total = prob.batch * prob.hq * NB
+    scale = units_total / len(blocks)
+    return {"value": dt * scale * 1e3, "unit": "ms/layer", "cores": cores, "kind": "oracle",
+            "sample": f"1 of {prob.hq} query heads x {len(blocks)} of {NB} query blocks "
+                      f"(every {step}th), {dt:.1f} s measured, scaled x{scale:.0f}"}
+
+
+# ----------------------------------------------------------------- main arm
+def run_ours(args, rank: int, world: int, local: int) -> None:
+    from block_sparse_long_score_b200 import (xattn_score, xattn_select, xattn_sparse_attn,
+                                              xattn_get_device_status,
+                                              xattn_score_workspace_bytes,
+                                              xattn_attn_workspace_bytes, make_shape)
+    from block_sparse_long_score_b200.synth import make_problem
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    prob = make_problem(WORKLOAD)
+    Qh, Kh, Vh = prob.Q.pin_memory(), prob.K.pin_memory(), prob.V.pin_memory()
+    Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
+    shape = make_shape(prob.batch, prob.hq, prob.hkv, prob.L, prob.d, prob.B, prob.S,
+                       prob.causal, "bf16")
+    NB = prob.NB
+    probs = torch.empty(prob.batch, prob.hq, NB, NB, device=dev, dtype=torch.float32)
+    ws_s = torch.empty(xattn_score_workspace_bytes(shape), device=dev, dtype=torch.uint8)
+    ws_a = torch.empty(xattn_attn_workspace_bytes(shape), device=dev, dtype=torch.uint8)
+    W = (NB + 31) // 32
+    mask = torch.empty(prob.batch, prob.hq, NB, W, device=dev, dtype=torch.int32)
+    counts = torch.empty(prob.batch, prob.hq, NB, device=dev, dtype=torch.int32)
+    idx = torch.empty(prob.batch, prob.hq, NB, NB, device=dev, dtype=torch.int32)
+    out = torch.empty_like(Q)
+    taus = prob.tau.tolist()
+    stream = torch.cuda.current_stream(dev)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        xattn_score(Q, K, prob.B, prob.S, prob.causal, probs=probs, workspace=ws_s)
+        if ev:
+            ev[1].record(stream)
+        xattn_select(probs, taus, prob.causal, out=(mask, counts, idx))
+        if ev:
+            ev[2].record(stream)
+        xattn_sparse_attn(Q, K, V, counts, idx, prob.B, prob.causal, out=out, workspace=ws_a)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if xattn_get_device_status(dev) != 0:
+        raise RuntimeError("device status reports a kernel time-out")
+    selected = int(counts.sum().item())
+    allowed = prob.batch * prob.hq * (NB * (NB + 1) // 2 if prob.causal else NB * NB)
+    density = selected / allowed
+
+    dist = world > 1
+    if dist:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    per = {"score": 0.0, "select": 0.0, "sparse_attn": 0.0}
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    for ev in evs:
+        per["score"] += ev[0].elapsed_time(ev[1])
+        per["select"] += ev[1].elapsed_time(ev[2])
+        per["sparse_attn"] += ev[2].elapsed_time(ev[3])
+    if dist:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    ms_step = total_ms / args.steps
+    if dist:
+        tt = torch.tensor([ms_step], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms_step = float(tt.item())
+    per = {k: v / args.steps for k, v in per.items()}
+
+    # end to end through the public API: pinned host -> device, the three calls,
+    # O -> pinned host, every step
+    Oh = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 3))
+    if dist:
+        torch.distributed.barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        Q.copy_(Qh, non_blocking=True)
+        K.copy_(Kh, non_blocking=True)
+        V.copy_(Vh, non_blocking=True)
+        step()
+        Oh.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist:
+        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    if xattn_get_device_status(dev) != 0:
+        raise RuntimeError("device status reports a kernel time-out")
+
+    pk = peaks()
+    attn_flops = 4.0 * prob.B * prob.B * prob.d * selected
+    attn_tflops = attn_flops / (per["sparse_attn"] * 1e-3) / 1e12
+    pairs = prob.hq * prob.batch * (NB * (NB + 1) // 2 if prob.causal else NB * NB)
+    score_flops = 2.0 * prob.B * prob.B * prob.d / prob.S * pairs
+    score_tflops = score_flops / (per["score"] * 1e-3) / 1e12
+    sel_bytes = 4.0 * pairs + 4.0 * selected + 4.0 * W * NB * prob.hq * prob.batch + \
+        4.0 * NB * prob.hq * prob.batch
+    sel_gbs = sel_bytes / (per["select"] * 1e-3) / 1e9
+    dense = dense_equiv_flops(prob)
+    dense_tflops = dense / (ms_step * 1e-3) / 1e12
+    peak_attn = pk["bf16_sustained"]
+    line = {
+        "metric": METRIC,
+        "value": ms_step / world,
+        "unit": "ms/layer",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded Llama-3.1-8B-shaped Q/K/V with planted sinks and slash bands)",
+        "config": workload_config(prob),
+        "dense_equiv_tflops": dense_tflops,
+        "pct_peak": 100.0 * dense_tflops / pk["bf16"],
+        "density": density,
+        "per_kernel_ms": per,
+        "score_select_share": (per["score"] + per["select"]) / ms_step,
+        "kernel_fracs": {
+            "score": {"tflops": score_tflops, "frac": score_tflops / pk["bf16_sustained"]},
+            "select": {"gbs": sel_gbs, "frac": sel_gbs / pk["hbm_gbs"]},
+            "sparse_attn": {"tflops": attn_tflops, "frac": attn_tflops / peak_attn},
+        },
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "attn_tc_kernel (xattn_sparse_attn; includes the LPT schedule kernel)",
+            "achieved": attn_tflops,
+            "peak": peak_attn,
+            "unit": "TFLOP/s",
+            "frac": attn_tflops / peak_attn,
+            "traffic": None,
+            "peak_source": f"{pk['source']} bf16 sustained (kernel timed inside a long step)",
+        },
+        "e2e": {
+            "value": e2e_ms / world,
+            "unit": "ms/layer",
+            "h2d_bytes_per_step": int(Q.numel() * 2 + K.numel() * 2 + V.numel() * 2),
+            "d2h_bytes_per_step": int(out.numel() * 2),
+        },
+        "gpu_launches": 5 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample(prob)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args, rank: int, world: int) -> None:
+    """The oracle on the host cores: a bounded sample of the same workload per
+    step, in the same unit."""
+    if rank != 0:
+        return
+    from block_sparse_long_score_b200.synth import make_problem
+    prob = make_problem(WORKLOAD)
+    for _ in range(args.warmup):
+        pass   # the oracle has no state to warm
+    vals = []
+    cb = None
+    steps = max(1, min(args.steps, 2))
+    for _ in range(steps):
+        cb = oracle_sample(prob, n_blocks=16)
+        vals.append(cb["value"])
+    v = float(np.mean(vals))
+    cb["value"] = v
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": v, "unit": "ms/layer", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(prob),
+        "cpu_baseline": cb,
+        "e2e": {"value": v, "unit": "ms/layer", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    try:
+        run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,79 @@
+// common.cuh -- shapes, workspace layout and launcher declarations shared by
+// the kernels and the C-ABI layer.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/xattn.h"
+
+namespace xattn {
+
+// Device status codes written into the per-device status word.
+constexpr int kStatusTimeout = 1;
+
+struct Dims {
+  int batch, hq, hkv, L, d, B, S, causal, dtype;
+  int NB, r, R, group;  // L/B, B/S, L/S, hq/hkv
+};
+
+// Partial log-sum-exp workspace of the scoring step.
+//
+// For every (batch, query head) there is one fp32 entry per (reshaped query
+// row rho, allowed key block j): log2 of the sum over the reshaped columns c
+// of block j of 2^(x[rho, c] * log2(e)), with x the scaled reshaped logits.
+// Causal rows of query block b = rho / r keep only j <= b, packed
+// row after row. Non-causal rows keep all NB entries.
+__host__ __device__ inline size_t part_head_elems(int NB, int r, int R, bool causal) {
+  return causal ? static_cast<size_t>(r) * NB * (NB + 1) / 2
+                : static_cast<size_t>(R) * NB;
+}
+
+__host__ __device__ inline size_t part_row_offset(int rho, int r, int NB, bool causal) {
+  if (!causal) return static_cast<size_t>(rho) * NB;
+  const size_t b = static_cast<size_t>(rho / r);
+  const size_t t = static_cast<size_t>(rho % r);
+  return static_cast<size_t>(r) * b * (b + 1) / 2 + t * (b + 1);
+}
+
+// ------------------------------------------------------------ launchers
+// Each returns cudaSuccess or the launch error. All are asynchronous.
+
+// bf16 tensor-core scoring GEMM: partials for every (bh, rho, allowed j).
+cudaError_t launch_score_tc(const Dims& D, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                            float* part, int* status, int num_sms, cudaStream_t st);
+
+// fp32 CUDA-core scoring, same partial layout.
+cudaError_t launch_score_simt(const Dims& D, const float* Q, const float* K, float* part,
+                              cudaStream_t st);
+
+// partials -> block probabilities P [bh, NB, NB].
+cudaError_t launch_score_reduce(const Dims& D, const float* part, float* probs,
+                                cudaStream_t st);
+
+struct TauArg {
+  float v[XATTN_MAX_HEADS];
+};
+
+// find_blocks on every row of P.
+cudaError_t launch_select(const Dims& D, const float* probs, const TauArg& tau, uint32_t* mask,
+                          int32_t* counts, int32_t* idx, cudaStream_t st);
+
+// Longest-list-first order of the work units (bh, b) into `order`.
+cudaError_t launch_sched(const Dims& D, const int32_t* counts, uint32_t* order,
+                         cudaStream_t st);
+
+// bf16 tensor-core block-sparse attention.
+cudaError_t launch_attn_tc(const Dims& D, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                           const CUtensorMap& tmV, const int32_t* counts, const int32_t* idx,
+                           const uint32_t* order, void* O, float* lse, int* status,
+                           int num_sms, cudaStream_t st);
+
+// fp32 CUDA-core block-sparse attention.
+cudaError_t launch_attn_simt(const Dims& D, const float* Q, const float* K, const float* V,
+                             const int32_t* counts, const int32_t* idx, float* O, float* lse,
+                             cudaStream_t st);
+
+}  // namespace xattn

@@ -1,0 +1,213 @@
+"""Python binding of libxattn.so: argument marshalling only.
+
+Every function here has the name of the C entry point it calls
+(``include/xattn.h``). It checks that the tensors are CUDA, contiguous and of
+the right dtype, allocates outputs and workspace with torch when the caller
+gives none, and passes raw pointers plus the current CUDA stream to the
+library. All computation happens in the library's CUDA kernels. There is no
+fallback: if the library is missing, or a call fails, this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = [
+    "XattnError", "xattn_score", "xattn_select", "xattn_sparse_attn",
+    "xattn_score_workspace_bytes", "xattn_attn_workspace_bytes",
+    "xattn_get_device_status", "xattn_strerror", "make_shape", "library_path",
+    "EXPORTED_SYMBOLS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIBNAME = "libxattn.so"
+
+XATTN_F32, XATTN_BF16 = 0, 1
+EXPORTED_SYMBOLS = (
+    "xattn_score_workspace_bytes", "xattn_score", "xattn_select",
+    "xattn_attn_workspace_bytes", "xattn_sparse_attn", "xattn_get_device_status",
+    "xattn_strerror",
+)
+
+
+class XattnError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {xattn_strerror(code)} ({code})")
+        self.code = code
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in
+                ("batch", "hq", "hkv", "L", "d", "B", "S", "causal", "dtype")]
+
+
+_lib_handle = None
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIBNAME)
+
+
+def _lib() -> ctypes.CDLL:
+    global _lib_handle
+    if _lib_handle is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise ImportError(
+                f"{path} is missing: build it with `python -m block_sparse_long_score_b200.build`")
+        lib = ctypes.CDLL(path)
+        vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+        sp = ctypes.POINTER(_Shape)
+        lib.xattn_score_workspace_bytes.argtypes = [sp]
+        lib.xattn_score_workspace_bytes.restype = sz
+        lib.xattn_attn_workspace_bytes.argtypes = [sp]
+        lib.xattn_attn_workspace_bytes.restype = sz
+        lib.xattn_score.argtypes = [vp, vp, sp, vp, vp, sz, vp]
+        lib.xattn_score.restype = i32
+        lib.xattn_select.argtypes = [vp, ctypes.POINTER(ctypes.c_float), sp, vp, vp, vp, vp]
+        lib.xattn_select.restype = i32
+        lib.xattn_sparse_attn.argtypes = [vp, vp, vp, sp, vp, vp, vp, vp, vp, sz, vp]
+        lib.xattn_sparse_attn.restype = i32
+        lib.xattn_get_device_status.argtypes = [vp]
+        lib.xattn_get_device_status.restype = i32
+        lib.xattn_strerror.argtypes = [i32]
+        lib.xattn_strerror.restype = ctypes.c_char_p
+        _lib_handle = lib
+    return _lib_handle
+
+
+def xattn_strerror(code: int) -> str:
+    return _lib().xattn_strerror(int(code)).decode()
+
+
+def make_shape(batch: int, hq: int, hkv: int, L: int, d: int, B: int, S: int, causal: bool,
+               dtype) -> _Shape:
+    dt = XATTN_BF16 if dtype in (torch.bfloat16, "bf16", XATTN_BF16) else XATTN_F32
+    return _Shape(int(batch), int(hq), int(hkv), int(L), int(d), int(B), int(S),
+                  1 if causal else 0, dt)
+
+
+def _shape_of(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal: bool) -> _Shape:
+    if Q.dim() != 4 or K.dim() != 4:
+        raise ValueError("Q and K must be [batch, heads, L, d]")
+    b, hq, L, d = Q.shape
+    if K.shape[0] != b or K.shape[2] != L or K.shape[3] != d:
+        raise ValueError("K shape does not match Q")
+    return make_shape(b, hq, K.shape[1], L, d, B, S, causal, Q.dtype)
+
+
+def _check(t: torch.Tensor, name: str, dtype=None) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _raise(fn: str, rc: int) -> None:
+    if rc != 0:
+        raise XattnError(fn, rc)
+
+
+def xattn_score_workspace_bytes(shape: _Shape) -> int:
+    return int(_lib().xattn_score_workspace_bytes(ctypes.byref(shape)))
+
+
+def xattn_attn_workspace_bytes(shape: _Shape) -> int:
+    return int(_lib().xattn_attn_workspace_bytes(ctypes.byref(shape)))
+
+
+def xattn_score(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal: bool,
+                probs: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Block probabilities P [batch, hq, L/B, L/B] (fp32) of antidiagonal scoring."""
+    _check(Q, "Q")
+    _check(K, "K", Q.dtype)
+    shape = _shape_of(Q, K, B, S, causal)
+    NB = shape.L // max(shape.B, 1)
+    if probs is None:
+        probs = torch.empty(shape.batch, shape.hq, NB, NB, device=Q.device, dtype=torch.float32)
+    _check(probs, "probs", torch.float32)
+    need = xattn_score_workspace_bytes(shape)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
+    _check(workspace, "workspace")
+    rc = _lib().xattn_score(Q.data_ptr(), K.data_ptr(), ctypes.byref(shape), probs.data_ptr(),
+                            workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                            _stream(Q.device))
+    _raise("xattn_score", rc)
+    return probs
+
+
+def xattn_select(probs: torch.Tensor, tau: Sequence[float], causal: bool,
+                 out: Optional[tuple] = None):
+    """find_blocks on every row of P. Returns (mask uint32 [.., NB, ceil(NB/32)] as
+    int32, counts int32 [.., NB], idx int32 [.., NB, NB])."""
+    _check(probs, "probs", torch.float32)
+    b, hq, NB, NB2 = probs.shape
+    if NB != NB2:
+        raise ValueError("probs must be [batch, hq, NB, NB]")
+    taus = [float(t) for t in tau]
+    if len(taus) != hq:
+        raise ValueError("tau needs one value per query head")
+    shape = make_shape(b, hq, hq, NB, 128, 1, 1, causal, XATTN_F32)
+    W = (NB + 31) // 32
+    if out is None:
+        mask = torch.empty(b, hq, NB, W, device=probs.device, dtype=torch.int32)
+        counts = torch.empty(b, hq, NB, device=probs.device, dtype=torch.int32)
+        idx = torch.empty(b, hq, NB, NB, device=probs.device, dtype=torch.int32)
+    else:
+        mask, counts, idx = out
+    for t, n in ((mask, "mask"), (counts, "counts"), (idx, "idx")):
+        _check(t, n, torch.int32)
+    tarr = (ctypes.c_float * hq)(*taus)
+    rc = _lib().xattn_select(probs.data_ptr(), tarr, ctypes.byref(shape), mask.data_ptr(),
+                             counts.data_ptr(), idx.data_ptr(), _stream(probs.device))
+    _raise("xattn_select", rc)
+    return mask, counts, idx
+
+
+def xattn_sparse_attn(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, counts: torch.Tensor,
+                      idx: torch.Tensor, B: int, causal: bool, out: Optional[torch.Tensor] = None,
+                      lse: Optional[torch.Tensor] | bool = None,
+                      workspace: Optional[torch.Tensor] = None):
+    """Attention over the listed key blocks. Returns O, or (O, lse) if lse is
+    True or a tensor."""
+    _check(Q, "Q")
+    _check(K, "K", Q.dtype)
+    _check(V, "V", Q.dtype)
+    _check(counts, "counts", torch.int32)
+    _check(idx, "idx", torch.int32)
+    shape = _shape_of(Q, K, B, 1, causal)
+    if out is None:
+        out = torch.empty_like(Q)
+    _check(out, "O", Q.dtype)
+    want_lse = lse is not None and lse is not False
+    if lse is True:
+        lse = torch.empty(Q.shape[:3], device=Q.device, dtype=torch.float32)
+    if want_lse:
+        _check(lse, "lse", torch.float32)
+    need = xattn_attn_workspace_bytes(shape)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
+    _check(workspace, "workspace")
+    rc = _lib().xattn_sparse_attn(Q.data_ptr(), K.data_ptr(), V.data_ptr(), ctypes.byref(shape),
+                                  counts.data_ptr(), idx.data_ptr(), out.data_ptr(),
+                                  lse.data_ptr() if want_lse else None, workspace.data_ptr(),
+                                  workspace.numel() * workspace.element_size(),
+                                  _stream(Q.device))
+    _raise("xattn_sparse_attn", rc)
+    return (out, lse) if want_lse else out
+
+
+def xattn_get_device_status(device=None) -> int:
+    """Synchronises the current stream; returns the device status (0 = ok)."""
+    return int(_lib().xattn_get_device_status(_stream(device)))

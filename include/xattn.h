@@ -1,0 +1,154 @@
+/*
+ * xattn.h -- C ABI of the XAttention prefill hot path on NVIDIA B200 (sm_100a).
+ *
+ * The three calls below are the three steps of "XAttention: Block Sparse
+ * Attention with Antidiagonal Scoring":
+ *   xattn_score        strided antidiagonal scoring and block probabilities
+ *                      (§2.1 Importance Prediction; §2.2; Algorithm 1)
+ *   xattn_select       find_blocks threshold selection per query-block row
+ *                      (§2.2 Threshold Block Selection, the find_blocks formula)
+ *   xattn_sparse_attn  attention over the selected blocks only
+ *                      (§1 step 3, "Block Sparse Attention")
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *   never allocates or frees them. Scratch space ("workspace") is also passed
+ *   in by the caller, sized by the *_workspace_bytes() query.
+ * - Q, K, V, O are contiguous [batch, heads, L, d] arrays. Q and O have hq
+ *   heads; K and V have hkv heads. hq must be a multiple of hkv, and query
+ *   head h reads KV head h / (hq / hkv) (grouped-query attention).
+ * - NB = L / B query blocks and key blocks. r = B / S reshaped rows per block.
+ * - Every call is asynchronous on the given CUDA stream (a cudaStream_t passed
+ *   as void*; NULL means the legacy default stream). No call synchronises the
+ *   device, except xattn_get_device_status.
+ * - Arguments are checked on the host before anything is launched. A failed
+ *   check returns a negative xattn_status and launches nothing.
+ * - Device-side faults that a kernel can detect on its own (a pipeline wait
+ *   that exceeded its time limit) are recorded in a per-device status word
+ *   that xattn_get_device_status reads and clears. Kernels never trap.
+ *
+ * Data types: XATTN_BF16 runs the tensor-core (tcgen05) kernels and needs
+ * d = 128 and B = 128. XATTN_F32 runs plain FP32 CUDA-core kernels for small
+ * problems and needs d in {32, 64, 128} and B <= 256.
+ */
+#ifndef XATTN_H_
+#define XATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  XATTN_OK = 0,
+  XATTN_ERR_INVALID_ARG = -1, /* bad shape, pointer, tau or stride */
+  XATTN_ERR_UNSUPPORTED = -2, /* valid, but outside what the kernels handle */
+  XATTN_ERR_CUDA = -3,        /* a CUDA runtime call failed */
+  XATTN_ERR_WORKSPACE = -4,   /* workspace pointer NULL or too small */
+  XATTN_ERR_TIMEOUT = -5      /* a kernel's bounded wait ran out (device status) */
+} xattn_status;
+
+typedef enum { XATTN_F32 = 0, XATTN_BF16 = 1 } xattn_dtype;
+
+/* Problem shape. causal != 0 selects causal attention. dtype is an xattn_dtype. */
+typedef struct {
+  int batch, hq, hkv, L, d, B, S, causal, dtype;
+} xattn_shape;
+
+/* Largest hq accepted (the per-head tau vector travels as a kernel argument). */
+#define XATTN_MAX_HEADS 256
+/* Largest NB = L / B accepted by xattn_select and xattn_score. */
+#define XATTN_MAX_BLOCKS 4096
+
+/*
+ * Bytes of workspace xattn_score needs: one fp32 partial log-sum-exp per
+ * (reshaped query row, allowed key block). Causal: batch*hq*r*NB*(NB+1)/2
+ * floats; non-causal: batch*hq*(L/S)*NB floats. Returns 0 for an invalid shape.
+ */
+size_t xattn_score_workspace_bytes(const xattn_shape* shape);
+
+/*
+ * Block probabilities P (§2.2; Algorithm 1's A_approx, block-summed).
+ *
+ * For each (batch, query head h, query block b), the reshaped queries are
+ * rows [Q[bB+tS+S-1], ..., Q[bB+tS]] (t = 0..r-1, joined along features),
+ * and the reshaped keys are rows [K[cS], ..., K[cS+S-1]]. Let
+ * x = Q_r K_r^T / sqrt(d*S). With causal != 0, reshaped column c is visible
+ * to global reshaped row rho only when c <= rho. A = row softmax of x.
+ * Then P[b, j] = (1/r) * (sum of A over the r x r sub-block (b, j)), so every
+ * row of P sums to 1. Causal rows are 0 for j > b.
+ *
+ * Q: [batch, hq, L, d], K: [batch, hkv, L, d], both of type shape->dtype and
+ *    16-byte aligned.
+ * probs: out, fp32 [batch, hq, NB, NB], fully written.
+ * ws / ws_bytes: workspace of at least xattn_score_workspace_bytes(shape).
+ * Errors: INVALID_ARG (NULL pointer, bad shape), UNSUPPORTED (dtype limits,
+ * NB > XATTN_MAX_BLOCKS), WORKSPACE, CUDA.
+ */
+int xattn_score(const void* Q, const void* K, const xattn_shape* shape, float* probs,
+                void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * find_blocks (§2.2): for every row (batch, h, b) of P, the smallest set of
+ * allowed key blocks whose probabilities sum to at least tau[h]. Blocks are
+ * ranked by probability (descending), ties by block index (ascending). The
+ * allowed blocks are 0..b when causal, all NB otherwise. If tau[h] >= 1, or the
+ * row's allowed sum never reaches tau[h], every allowed block is selected.
+ * Sums are accumulated in fp64.
+ *
+ * probs: fp32 [batch, hq, NB, NB], device.
+ * tau:   HOST pointer to hq floats, each in (0, 1]; INVALID_ARG otherwise.
+ * mask:   out, uint32 [batch, hq, NB, ceil(NB/32)]; bit (j % 32) of word j / 32
+ *         is set iff block j is selected. Fully written.
+ * counts: out, int32 [batch, hq, NB], the number of selected blocks.
+ * idx:    out, int32 [batch, hq, NB, NB]; the first counts[...] entries of a
+ *         row are the selected block indices in ascending order. The rest of
+ *         the row is left unwritten.
+ */
+int xattn_select(const float* probs, const float* tau, const xattn_shape* shape,
+                 uint32_t* mask, int32_t* counts, int32_t* idx, void* stream);
+
+/*
+ * Bytes of workspace xattn_sparse_attn needs (the work schedule:
+ * 4 * (batch*hq*NB + 64) bytes). Returns 0 for an invalid shape.
+ */
+size_t xattn_attn_workspace_bytes(const xattn_shape* shape);
+
+/*
+ * Block-sparse attention. For each query q in query block b of head h:
+ *   O[q] = sum_k softmax_k(Q[q] . K[k] / sqrt(d)) V[k]
+ * over the keys k of the blocks idx[batch, h, b, 0 .. counts[batch, h, b]-1]
+ * (KV head h / (hq/hkv)). With causal != 0, keys k > q are dropped, and listed
+ * blocks j > b are skipped. A row with no visible key gets O = 0 and
+ * lse = -inf.
+ *
+ * Q, K, V: as for xattn_score (16-byte aligned); O: out, same type as Q,
+ *          [batch, hq, L, d].
+ * counts, idx: as written by xattn_select (device).
+ * lse: out, optional (may be NULL), fp32 [batch, hq, L], natural-log
+ *      log-sum-exp of each row's scaled logits.
+ * ws / ws_bytes: at least xattn_attn_workspace_bytes(shape).
+ * The work units (batch, h, b) run longest-list-first on persistent CTAs.
+ */
+int xattn_sparse_attn(const void* Q, const void* K, const void* V, const xattn_shape* shape,
+                      const int32_t* counts, const int32_t* idx, void* O, float* lse,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's status
+ * word. Returns XATTN_OK, XATTN_ERR_TIMEOUT if a kernel gave up a bounded
+ * wait since the last call, or XATTN_ERR_CUDA if the stream reports an error.
+ */
+int xattn_get_device_status(void* stream);
+
+/* Static, human-readable text for an xattn_status value. */
+const char* xattn_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* XATTN_H_ */

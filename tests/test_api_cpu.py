@@ -1,0 +1,93 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+that include/xattn.h declares, sizes its workspaces, and rejects bad
+arguments on the host before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_long_score_b200 import build as xbuild
+from block_sparse_long_score_b200 import xattn as X
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = ctypes.c_void_p(0x10000)   # never dereferenced: every call below fails its host checks
+
+
+@pytest.fixture(scope="module")
+def lib():
+    xbuild.build()
+    return X._lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "xattn.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(xattn_\w+)\s*\(", src, re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(X.EXPORTED_SYMBOLS)
+
+
+def test_workspace_sizes(lib):
+    s = X.make_shape(1, 32, 8, 131072, 128, 128, 16, True, "bf16")
+    NB, r = 1024, 8
+    assert X.xattn_score_workspace_bytes(s) == 32 * r * NB * (NB + 1) // 2 * 4 + 256
+    assert X.xattn_attn_workspace_bytes(s) == 4 * (32 * NB + 64)
+    nc = X.make_shape(1, 24, 24, 76800, 128, 128, 4, False, "bf16")
+    assert X.xattn_score_workspace_bytes(nc) == 24 * (76800 // 4) * 600 * 4 + 256
+    bad = X.make_shape(1, 32, 8, 1000, 128, 128, 16, True, "bf16")
+    assert X.xattn_score_workspace_bytes(bad) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(L=1000), -1),             # L % B != 0
+    (dict(S=3), -1),                # B % S != 0
+    (dict(hkv=3), -1),              # hq % hkv != 0
+    (dict(d=64), -2),               # bf16 needs d = 128
+    (dict(B=64, S=8), -2),          # bf16 needs B = 128
+    (dict(hq=512, hkv=8), -2),      # too many heads
+    (dict(L=128 * 8192), -2),       # NB above the maximum
+])
+def test_bad_shapes_rejected(lib, kw, code):
+    a = dict(batch=1, hq=32, hkv=8, L=4096, d=128, B=128, S=8, causal=True, dtype="bf16")
+    a.update(kw)
+    s = X.make_shape(**a)
+    rc = lib.xattn_score(FAKE, FAKE, ctypes.byref(s), FAKE, FAKE, 1 << 40, None)
+    assert rc == code
+    rc = lib.xattn_sparse_attn(FAKE, FAKE, FAKE, ctypes.byref(s), FAKE, FAKE, FAKE, None,
+                               FAKE, 1 << 40, None)
+    assert rc == code
+
+
+def test_null_pointers_and_workspace(lib):
+    s = X.make_shape(1, 4, 2, 1024, 128, 128, 8, True, "bf16")
+    assert lib.xattn_score(None, FAKE, ctypes.byref(s), FAKE, FAKE, 1 << 40, None) == -1
+    assert lib.xattn_score(FAKE, FAKE, ctypes.byref(s), FAKE, None, 1 << 40, None) == -4
+    assert lib.xattn_score(FAKE, FAKE, ctypes.byref(s), FAKE, FAKE, 16, None) == -4
+    assert lib.xattn_sparse_attn(FAKE, FAKE, FAKE, ctypes.byref(s), FAKE, FAKE, FAKE, None,
+                                 FAKE, 8, None) == -4
+    assert lib.xattn_score(FAKE, FAKE, None, FAKE, FAKE, 1 << 40, None) == -1
+
+
+@pytest.mark.parametrize("tau", [0.0, -0.5, 1.5, float("nan")])
+def test_tau_out_of_range(lib, tau):
+    s = X.make_shape(1, 2, 2, 1024, 128, 128, 8, True, "bf16")
+    t = (ctypes.c_float * 2)(0.9, tau)
+    assert lib.xattn_select(FAKE, t, ctypes.byref(s), FAKE, FAKE, FAKE, None) == -1
+
+
+def test_misaligned_bf16_pointer(lib):
+    s = X.make_shape(1, 4, 2, 1024, 128, 128, 8, True, "bf16")
+    odd = ctypes.c_void_p(0x10008)
+    assert lib.xattn_score(odd, FAKE, ctypes.byref(s), FAKE, FAKE, 1 << 40, None) == -1
+
+
+def test_strerror(lib):
+    assert X.xattn_strerror(0) == "ok"
+    assert "timed out" in X.xattn_strerror(-5)
+    assert X.xattn_strerror(42) == "unknown status"
