@@ -84,7 +84,7 @@ __device__ __forceinline__ void decode_tile(long long t, const Params& p, int& b
 // blocks; for RP > 32 a block spans RP/32 chunks and (m, s) carry across.
 template <int RP>
 __device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], int c0, int rho,
-                                               int R, int jmax, bool need_mask,
+                                               int R, int jmax, bool need_mask, bool causal,
                                                float sl2, float* prow, float& m_run,
                                                float& s_run) {
   float x[32];
@@ -93,7 +93,7 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], int c0, 
     float a = __uint_as_float(v[i]);
     if (need_mask) {
       const int c = c0 + i;
-      if (c >= R || c > rho) a = -INFINITY;
+      if (c >= R || (causal && c > rho)) a = -INFINITY;
     }
     x[i] = a;
   }
@@ -105,6 +105,10 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], int c0, 
       float m = -INFINITY;
 #pragma unroll
       for (int i = 0; i < RP; ++i) m = fmaxf(m, x[g * RP + i]);
+      if (m == -INFINITY) {  // no visible column (cannot happen for j <= jmax)
+        prow[j] = -INFINITY;
+        continue;
+      }
       const float mb = m * sl2;
       float s = 0.f;
 #pragma unroll
@@ -149,7 +153,8 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tacc, int rho, int n0, co
     tmem_ld_wait();
     const int c0 = n0 + ch * 32;
     if (row_ok && c0 < p.R && (c0 / RP) <= jmax) {
-      epilogue_chunk<RP>(v, c0, rho, p.R, jmax, need_mask, p.scale_log2, prow, m_run, s_run);
+      epilogue_chunk<RP>(v, c0, rho, p.R, jmax, need_mask, p.causal != 0, p.scale_log2, prow,
+                         m_run, s_run);
     }
   }
 }

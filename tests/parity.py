@@ -36,6 +36,8 @@ def lists_from(counts: np.ndarray, idx: np.ndarray, bb: int, h: int, blocks) -> 
 
 def check_probs(P_gpu: np.ndarray, P_ref: np.ndarray) -> float:
     """Returns the worst ratio of |error| to the allowed bound (<= 1 passes)."""
+    if not np.all(np.isfinite(P_gpu)):
+        return float("inf")
     err = np.abs(P_gpu.astype(np.float64) - P_ref)
     bound = P_RTOL * np.abs(P_ref) + P_ATOL
     return float(np.max(err / bound))
