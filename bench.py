@@ -31,7 +31,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "prefill attn ms/layer at 128K (score+select+sparse); dense-equiv TFLOP/s, %peak"
-WORKLOAD = "c2"
+WORKLOAD = "c2"   # the 128K Llama-shaped layer the metric is quoted on
 
 
 def peaks() -> dict:
@@ -143,6 +143,14 @@ def oracle_sample(prob, n_blocks: int = 48) -> dict:
                       f"(every {step}th), {dt:.1f} s measured, scaled x{scale:.0f}"}
 
 
+def problem_overrides(args) -> dict:
+    """--heads N keeps N query heads (and the same 4:1 GQA ratio) of the
+    workload: a smaller case of the same kernels, for ncu captures."""
+    if not args.heads:
+        return {}
+    return {"hq": args.heads, "hkv": max(1, args.heads // 4)}
+
+
 # ----------------------------------------------------------------- main arm
 def run_ours(args, rank: int, world: int, local: int) -> None:
     from block_sparse_long_score_b200 import (xattn_score, xattn_select, xattn_sparse_attn,
@@ -152,7 +160,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     from block_sparse_long_score_b200.synth import make_problem
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    prob = make_problem(WORKLOAD)
+    prob = make_problem(WORKLOAD, **problem_overrides(args))
     Qh, Kh, Vh = prob.Q.pin_memory(), prob.K.pin_memory(), prob.V.pin_memory()
     Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
     shape = make_shape(prob.batch, prob.hq, prob.hkv, prob.L, prob.d, prob.B, prob.S,
@@ -314,7 +322,7 @@ def run_reference(args, rank: int, world: int) -> None:
     if rank != 0:
         return
     from block_sparse_long_score_b200.synth import make_problem
-    prob = make_problem(WORKLOAD)
+    prob = make_problem(WORKLOAD, **problem_overrides(args))
     for _ in range(args.warmup):
         pass   # the oracle has no state to warm
     vals = []
@@ -345,6 +353,8 @@ def main() -> None:
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="profiling case: keep this many query heads (default: all 32)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

@@ -128,14 +128,13 @@ def _tiny(cfg: dict, L: int, seed: int) -> tuple:
     return Q, K, V, recipe
 
 
-def _llama(cfg: dict, L: int, hq: int, hkv: int, seed: int) -> tuple:
+def _llama(cfg: dict, L: int, hq: int, hkv: int, seed: int, gamma: float) -> tuple:
     g = torch.Generator().manual_seed(seed)
     d, batch = cfg["d"], cfg["batch"]
     dt = cfg["dtype"]
     gsz = hq // hkv
     w = 512
     nb = cfg["bands"]
-    gamma = SLASH_GAMMA
     beta = math.sqrt(15.0 * d)   # |k_sink| ~ sqrt(d + beta^2) = 4 sqrt(d)
     # Per KV group: sink direction and band offsets.
     u = [_unit(g, d) for _ in range(hkv)]
@@ -199,7 +198,7 @@ def _video(cfg: dict, frames: int, frame_tokens: int, hq: int, seed: int) -> tup
 def make_problem(name: str, *, L: int | None = None, hq: int | None = None,
                  hkv: int | None = None, S: int | None = None, frames: int | None = None,
                  frame_tokens: int | None = None, seed: int | None = None,
-                 tau: float | None = None) -> Problem:
+                 tau: float | None = None, gamma: float | None = None) -> Problem:
     """Build one workload by name ("c0".."c4").
 
     The keyword overrides shrink a workload for tests: same recipe, fewer
@@ -220,7 +219,8 @@ def make_problem(name: str, *, L: int | None = None, hq: int | None = None,
         Q, K, V, recipe = _tiny(cfg, L, seed)
     elif cfg["kind"] == "llama":
         L = cfg["L"] if L is None else L
-        Q, K, V, recipe = _llama(cfg, L, hq, hkv, seed)
+        Q, K, V, recipe = _llama(cfg, L, hq, hkv, seed,
+                                 SLASH_GAMMA if gamma is None else gamma)
     else:
         fr = cfg["frames"] if frames is None else frames
         ft = cfg["frame_tokens"] if frame_tokens is None else frame_tokens
