@@ -9,6 +9,6 @@ calls raise if it is missing.
 from .xattn import (  # noqa: F401
     XattnError, xattn_score, xattn_select, xattn_sparse_attn, xattn_score_workspace_bytes,
     xattn_attn_workspace_bytes, xattn_get_device_status, xattn_strerror, make_shape,
-    library_path, EXPORTED_SYMBOLS,
+    library_path, EXPORTED_SYMBOLS, xattn_sparse_attn_noalloc,
 )
 from .pipeline import prefill_attention  # noqa: F401

@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "host.cuh"
 
 namespace xattn {
 
@@ -15,15 +16,7 @@ namespace xattn {
 // kStatusTimeout here; xattn_get_device_status reads and clears it.
 __device__ int g_status_word;
 
-namespace {
-
-constexpr int kMaxDevices = 64;
-
-struct DeviceState {
-  bool ready = false;
-  int* status = nullptr;  // device address of g_status_word
-  int num_sms = 0;
-};
+namespace host {
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -132,10 +125,11 @@ int make_map_reshaped(CUtensorMap* m, const void* ptr, int S, int R, int bh, int
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? XATTN_OK : XATTN_ERR_CUDA; }
 
-}  // namespace
+}  // namespace host
 }  // namespace xattn
 
 using namespace xattn;
+using namespace xattn::host;
 
 extern "C" {
 

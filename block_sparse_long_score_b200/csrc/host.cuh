@@ -1,0 +1,31 @@
+// host.cuh -- host-side helpers of the C-ABI layer (argument checks, per-device
+// state, TMA descriptors), shared by the entry-point files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace xattn {
+namespace host {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  int* status = nullptr;  // device address of the status word
+  int num_sms = 0;
+};
+
+// State of the current device, created on first use. Returns an xattn_status.
+int device_state(DeviceState** out);
+// Checks a shape and fills the derived sizes. Returns an xattn_status.
+int check_shape(const xattn_shape* sh, Dims* D);
+bool aligned16(const void* p);
+// 2-D bf16 view [rows, 128] with 64 x 128 boxes and 128-byte swizzle.
+int make_map_2d(CUtensorMap* m, const void* ptr, long long rows);
+int cuda_status(cudaError_t e);
+
+}  // namespace host
+}  // namespace xattn

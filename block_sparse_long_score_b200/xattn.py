@@ -19,7 +19,7 @@ __all__ = [
     "XattnError", "xattn_score", "xattn_select", "xattn_sparse_attn",
     "xattn_score_workspace_bytes", "xattn_attn_workspace_bytes",
     "xattn_get_device_status", "xattn_strerror", "make_shape", "library_path",
-    "EXPORTED_SYMBOLS",
+    "EXPORTED_SYMBOLS", "xattn_sparse_attn_noalloc", "NOALLOC_MAX_UNITS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,8 +29,10 @@ XATTN_F32, XATTN_BF16 = 0, 1
 EXPORTED_SYMBOLS = (
     "xattn_score_workspace_bytes", "xattn_score", "xattn_select",
     "xattn_attn_workspace_bytes", "xattn_sparse_attn", "xattn_get_device_status",
-    "xattn_strerror",
+    "xattn_strerror", "xattn_sparse_attn_noalloc",
 )
+# batch * hq * (L / B) limit of xattn_sparse_attn_noalloc (XATTN_NOALLOC_MAX_UNITS)
+NOALLOC_MAX_UNITS = 1 << 18
 
 
 class XattnError(RuntimeError):
@@ -71,6 +73,8 @@ def _lib() -> ctypes.CDLL:
         lib.xattn_select.restype = i32
         lib.xattn_sparse_attn.argtypes = [vp, vp, vp, sp, vp, vp, vp, vp, vp, sz, vp]
         lib.xattn_sparse_attn.restype = i32
+        lib.xattn_sparse_attn_noalloc.argtypes = [vp, vp, vp, sp, vp, vp, vp, vp, vp]
+        lib.xattn_sparse_attn_noalloc.restype = i32
         lib.xattn_get_device_status.argtypes = [vp]
         lib.xattn_get_device_status.restype = i32
         lib.xattn_strerror.argtypes = [i32]
@@ -206,6 +210,30 @@ def xattn_sparse_attn(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, counts:
                                   _stream(Q.device))
     _raise("xattn_sparse_attn", rc)
     return (out, lse) if want_lse else out
+
+
+def xattn_sparse_attn_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                              counts: torch.Tensor, idx: torch.Tensor, B: int, causal: bool,
+                              out: torch.Tensor, lse: Optional[torch.Tensor] = None):
+    """xattn_sparse_attn for callers that cannot allocate: the library keeps the
+    work order in its own device array, and the caller passes every output
+    buffer (``out``, and ``lse`` if wanted). Nothing is allocated here."""
+    _check(Q, "Q")
+    _check(K, "K", Q.dtype)
+    _check(V, "V", Q.dtype)
+    _check(counts, "counts", torch.int32)
+    _check(idx, "idx", torch.int32)
+    _check(out, "O", Q.dtype)
+    if lse is not None:
+        _check(lse, "lse", torch.float32)
+    shape = _shape_of(Q, K, B, 1, causal)
+    rc = _lib().xattn_sparse_attn_noalloc(Q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                          ctypes.byref(shape), counts.data_ptr(),
+                                          idx.data_ptr(), out.data_ptr(),
+                                          lse.data_ptr() if lse is not None else None,
+                                          _stream(Q.device))
+    _raise("xattn_sparse_attn_noalloc", rc)
+    return out
 
 
 def xattn_get_device_status(device=None) -> int:

@@ -137,6 +137,34 @@ int xattn_sparse_attn(const void* Q, const void* K, const void* V, const xattn_s
                       const int32_t* counts, const int32_t* idx, void* O, float* lse,
                       void* ws, size_t ws_bytes, void* stream);
 
+/* Largest batch*hq*(L/B) accepted by xattn_sparse_attn_noalloc. */
+#define XATTN_NOALLOC_MAX_UNITS (1 << 18)
+
+/*
+ * xattn_sparse_attn without a workspace: the same attention, and for the same
+ * inputs the same outputs, but the call allocates nothing and takes no
+ * workspace. This entry point has no counterpart in the paper. It is for
+ * callers that cannot call cudaMalloc: a host program whose device memory all
+ * belongs to another allocator, or a serving loop that may not allocate once
+ * running (an allocation can synchronise the device or fail under memory
+ * pressure).
+ *
+ * The work order lives in a __device__ array of the library, sized for
+ * XATTN_NOALLOC_MAX_UNITS work units (1 MiB). Each GPU that loads the library
+ * holds it until the process exits. Returns XATTN_ERR_WORKSPACE when
+ * batch*hq*(L/B) exceeds that limit.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any
+ * stream capture. All calls on a device share the array and it keeps the last
+ * call's contents. Calls whose kernels overlap on the GPU (for example on two
+ * unordered streams) race on it, so order such calls on one stream.
+ * Arguments and other errors are as for xattn_sparse_attn.
+ */
+int xattn_sparse_attn_noalloc(const void* Q, const void* K, const void* V,
+                              const xattn_shape* shape, const int32_t* counts,
+                              const int32_t* idx, void* O, float* lse, void* stream);
+
 /*
  * Synchronises `stream`, then reads and clears the current device's status
  * word. Returns XATTN_OK, XATTN_ERR_TIMEOUT if a kernel gave up a bounded
