@@ -46,13 +46,17 @@ def peaks() -> dict:
 
 
 def workload_config(prob) -> dict:
+    kinds = {"c1": "llama3.1-8b attention layer", "c2": "llama3.1-8b attention layer",
+             "c3": "llama3.1-8b attention layer", "c4": "video-DiT attention layer (30x2560)"}
+    taus = sorted(set(np.round(prob.tau.astype(np.float64), 2).tolist()))
     return {
-        "workload": f"llama3.1-8b attention layer, L={prob.L}, hq={prob.hq}/hkv={prob.hkv}, "
-                    f"d={prob.d}, bf16, causal, B={prob.B}, S={prob.S}, "
-                    "tau per head from {0.8,0.85,0.9,0.95}",
+        "workload": f"{kinds.get(prob.name, prob.name)}, L={prob.L}, hq={prob.hq}/hkv={prob.hkv}, "
+                    f"d={prob.d}, {prob.dtype}, {'causal' if prob.causal else 'non-causal'}, "
+                    f"B={prob.B}, S={prob.S}, tau in {taus}",
         "L": prob.L, "hq": prob.hq, "hkv": prob.hkv, "d": prob.d, "B": prob.B, "S": prob.S,
         "causal": prob.causal, "global_batch": prob.batch,
-        "l2": "no flush: inputs (Q/K/V 1.5 GB) and scoring partials (0.54 GB) exceed the 126 MB L2",
+        "l2": "no flush: inputs (Q/K/V) exceed the 126 MB L2" if prob.Q.numel() * 2 > 126e6
+              else "inputs fit in L2 (small profiling case)",
         "parallelism": "replicas",
     }
 
@@ -162,11 +166,18 @@ def oracle_sample(prob, n_blocks: int = 48) -> dict:
 
 
 def problem_overrides(args) -> dict:
-    """--heads N keeps N query heads (and the same 4:1 GQA ratio) of the
-    workload: a smaller case of the same kernels, for ncu captures."""
-    if not args.heads:
-        return {}
-    return {"hq": args.heads, "hkv": max(1, args.heads // 4)}
+    """--heads N keeps N query heads (and the workload's GQA ratio): a smaller
+    case of the same kernels, for ncu captures. --stride picks the stride of
+    the video layer's sweep."""
+    from block_sparse_long_score_b200.synth import CONFIGS
+    cfg = CONFIGS[args.config]
+    kw = {}
+    if args.heads:
+        g = cfg["hq"] // cfg["hkv"]
+        kw.update(hq=args.heads, hkv=max(1, args.heads // g))
+    if args.stride:
+        kw["S"] = args.stride
+    return kw
 
 
 # ----------------------------------------------------------------- main arm
@@ -178,7 +189,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     from block_sparse_long_score_b200.synth import make_problem
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    prob = make_problem(WORKLOAD, **problem_overrides(args))
+    prob = make_problem(args.config, **problem_overrides(args))
     Qh, Kh, Vh = prob.Q.pin_memory(), prob.K.pin_memory(), prob.V.pin_memory()
     Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
     shape = make_shape(prob.batch, prob.hq, prob.hkv, prob.L, prob.d, prob.B, prob.S,
@@ -332,7 +343,7 @@ def run_reference(args, rank: int, world: int) -> None:
     if rank != 0:
         return
     from block_sparse_long_score_b200.synth import make_problem
-    prob = make_problem(WORKLOAD, **problem_overrides(args))
+    prob = make_problem(args.config, **problem_overrides(args))
     for _ in range(args.warmup):
         pass   # the oracle has no state to warm
     vals = []
@@ -363,6 +374,9 @@ def main() -> None:
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--config", default=WORKLOAD, choices=["c1", "c2", "c3", "c4"],
+                    help="workload (default c2, the 128K layer the metric is quoted on)")
+    ap.add_argument("--stride", type=int, default=0, help="stride S for the video layer (c4)")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling case: keep this many query heads (default: all 32)")
     args = ap.parse_args()

@@ -7,20 +7,31 @@
 // blocks (B = 128, d = 128). For each listed key block j:
 //   S_j = Q K_j^T                 tcgen05.mma, A = Q (smem), B = K_j (smem) -> TMEM
 //   P_j = exp2(S_j * c - m)       softmax warps, one TMEM lane (query row) each,
-//                                 online max with lazy rescaling of O
+//                                 running max with lazy rescaling of O
 //   O  += P_j V_j                 tcgen05.mma, A = P_j (TMEM, bf16), B = V_j (smem)
-// P_j is written back over the first 64 TMEM columns of S_j as packed bf16, so
-// a CTA needs 256 TMEM columns (S 128 + O 128). Two CTAs share an SM, and
-// the tensor core switches between them: one CTA's softmax overlaps the
-// other's MMAs.
+// P_j is written back over the first 64 TMEM columns of S_j as packed bf16.
 //
-// Warp roles (192 threads):
-//   warp 0      TMA producer: Q once per unit, then K_j, V_j into a 2-slot ring
-//   warp 1      TMEM allocator + MMA issuer
-//   warps 2..5  softmax and output epilogue (warp w owns TMEM lanes 32*(w%4)..)
-// Units come from the longest-list-first order, round-robin over the CTAs.
-// Every pipeline wait is bounded; on time-out the CTA raises its abort flag,
-// drains, frees TMEM and records XATTN_ERR_TIMEOUT in the status word.
+// One persistent CTA per SM runs two independent units at a time ("slots").
+// Each slot has its own Q tile in shared memory, its own 256 TMEM columns
+// (S 128 + O 128) and its own softmax warpgroup. One MMA thread interleaves
+// the slots -- S(0), S(1), then PV(0), S(0, next), PV(1), S(1, next), ... --
+// so the tensor core works on one slot while the other slot's softmax runs.
+// K_j and V_j stream through a 5-stage ring; the producer walks exactly the
+// same merged event order as the MMA thread, so the ring is a plain FIFO.
+//
+// Warp roles (384 threads, three warpgroups):
+//   warps 0..3  control warpgroup, 80 registers a thread: warp 0 TMA producer,
+//               warp 1 TMEM allocator + MMA issuer (warps 2, 3 idle)
+//   warps 4..7  softmax + output epilogue of slot 0, 208 registers a thread
+//   warps 8..11 softmax + output epilogue of slot 1 (warp w owns TMEM lanes
+//               32*(w%4) .. 32*(w%4)+31)
+// The launch gives 384 x 168 registers; setmaxnreg moves them from the
+// control warpgroup to the softmax warpgroups (128*80 + 256*208 <= 384*168),
+// which hold a whole 128-score row in registers.
+// Units come from the longest-list-first order: slot s of CTA c takes units
+// 2c+s, 2c+s+2G, ... (G = grid size). Every pipeline wait is bounded; on
+// time-out the CTA raises its abort flag, drains, frees TMEM and records
+// XATTN_ERR_TIMEOUT in the status word.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -29,18 +40,23 @@
 namespace xattn {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
 constexpr int kBlk = 128;                      // B (rows per query / key block)
 constexpr int kD = 128;                        // head dim
 constexpr int kHalf = kBlk * 64 * 2;           // one 64-feature box: 16 KB
 constexpr int kTileBytes = 2 * kHalf;          // 128 x 128 bf16: 32 KB
-constexpr int kStages = 2;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0;                  // S_j (fp32), P_j (bf16) aliases cols 0..63
-constexpr uint32_t kColO = 128;                // O accumulator (fp32)
+constexpr int kStages = 5;
+constexpr int kSlots = 2;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSlotCols = 256;            // per slot: S at +0 (P aliases +0..63), O at +128
+constexpr uint32_t kColO = 128;
 constexpr uint32_t kIdescS = idesc_bf16_f32(kBlk, kBlk, 0, 0);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(kBlk, kD, 0, 1);  // V is MN-major
 constexpr float kRescaleLog2 = 8.0f;           // rescale O only when the max grows by > 2^8
+constexpr int kLaunchRegs = 168;               // registers a thread at launch (__launch_bounds__)
+constexpr int kCtrlRegs = 80, kSoftmaxRegs = 208;
+static_assert(128 * kCtrlRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs,
+              "setmaxnreg split exceeds the registers the block is launched with");
 
 struct Params {
   int L, NB, hq, hkv, group, causal, units;
@@ -54,48 +70,255 @@ struct Params {
 };
 
 struct Smem {
-  uint64_t q_full, q_empty;
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full, p_full, pv_done, o_empty;
+  uint64_t q_full[kSlots], q_empty[kSlots];
+  uint64_t s_full[kSlots], p_full[kSlots], pv_done[kSlots], o_empty[kSlots];
   uint32_t tmem_base;
   int abort;
 };
 
-// Number of listed blocks a unit actually uses: causal lists drop the
-// trailing blocks above the diagonal (the list is ascending).
+// Walks the blocks of one slot's units in order, skipping units with no block.
+struct Cursor {
+  int k;        // position in the unit order
+  int step;     // distance between this slot's units (2 * grid)
+  int unit, bh, qb, n, j;
+  const int32_t* list;
+  bool valid;
+};
+
 __device__ __forceinline__ int effective_count(const Params& p, const int32_t* list, int n,
                                                int qb) {
   n = n < 0 ? 0 : (n > p.NB ? p.NB : n);
   if (!p.causal) return n;
-  while (n > 0 && list[n - 1] > qb) --n;
+  while (n > 0 && list[n - 1] > qb) --n;  // ascending list: drop blocks above the diagonal
   return n;
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+__device__ __forceinline__ void cursor_seek(Cursor& c, const Params& p) {
+  for (; c.k < p.units; c.k += c.step) {
+    c.unit = static_cast<int>(p.order[c.k]);
+    c.bh = c.unit / p.NB;
+    c.qb = c.unit % p.NB;
+    c.list = p.idx + static_cast<size_t>(c.unit) * p.NB;
+    c.n = effective_count(p, c.list, p.counts[c.unit], c.qb);
+    c.j = 0;
+    if (c.n > 0) {
+      c.valid = true;
+      return;
+    }
+  }
+  c.valid = false;
+}
+
+__device__ __forceinline__ void cursor_init(Cursor& c, const Params& p, int slot) {
+  c.k = 2 * blockIdx.x + slot;
+  c.step = 2 * gridDim.x;
+  cursor_seek(c, p);
+}
+
+// Moves past the current block; returns false when the slot has no more work.
+__device__ __forceinline__ bool cursor_next(Cursor& c, const Params& p) {
+  if (++c.j < c.n) return true;
+  c.k += c.step;
+  cursor_seek(c, p);
+  return c.valid;
+}
+
+
+struct SlotState {
+  Cursor cur;
+  bool pend;       // an S was issued whose PV is still to come
+  int pend_j;      // block index of that S within its unit
+  uint32_t units;  // units started (first S issued)
+  uint32_t blocks; // PV events done
+};
+
+struct Ring {
+  int stage;
+  uint32_t phase;
+  long long issued;
+  __device__ __forceinline__ void next() {
+    if (++stage == kStages) {
+      stage = 0;
+      phase ^= 1;
+    }
+  }
+};
+
+struct Ctx {
+  const Params* p;
+  Smem* sm;
+  uint8_t* q_smem;
+  uint8_t* kv_smem;
+  uint32_t tmem;
+  const CUtensorMap* tmQ;
+  const CUtensorMap* tmK;
+  const CUtensorMap* tmV;
+  volatile int* abort;
+};
+
+// S event of slot kSlot for the cursor's current block. The producer loads Q
+// (first block of a unit) and K; the MMA thread issues S = Q K^T.
+template <bool kMma, int kSlot>
+__device__ __forceinline__ bool event_s(SlotState& st, Ring& ring, const Ctx& x) {
+  const Params& p = *x.p;
+  Smem* sm = x.sm;
+  Cursor& c = st.cur;
+  const bool first = c.j == 0;
+  const bool last = c.j == c.n - 1;
+  if (!kMma) {
+    if (first) {
+      if (!mbar_wait(&sm->q_empty[kSlot], (st.units & 1) ^ 1, x.abort)) return false;
+      mbar_arrive_expect_tx(&sm->q_full[kSlot], kTileBytes);
+      const int qrow = c.bh * p.L + c.qb * kBlk;
+      tma_load_2d(x.q_smem + kSlot * kTileBytes, x.tmQ, &sm->q_full[kSlot], 0, qrow);
+      tma_load_2d(x.q_smem + kSlot * kTileBytes + kHalf, x.tmQ, &sm->q_full[kSlot], 64, qrow);
+    }
+    if (!mbar_wait(&sm->kv_empty[ring.stage], ring.phase ^ 1, x.abort)) return false;
+    const int kvbh = (c.bh / p.hq) * p.hkv + (c.bh % p.hq) / p.group;
+    const int krow = kvbh * p.L + c.list[c.j] * kBlk;
+    uint8_t* dst = x.kv_smem + ring.stage * kTileBytes;
+    mbar_arrive_expect_tx(&sm->kv_full[ring.stage], kTileBytes);
+    tma_load_2d(dst, x.tmK, &sm->kv_full[ring.stage], 0, krow);
+    tma_load_2d(dst + kHalf, x.tmK, &sm->kv_full[ring.stage], 64, krow);
+    ++ring.issued;
+  } else {
+    if (first && !mbar_wait(&sm->q_full[kSlot], st.units & 1, x.abort)) return false;
+    if (!mbar_wait(&sm->kv_full[ring.stage], ring.phase, x.abort)) return false;
+    tc_fence_after();
+    const uint32_t q_addr = smem_u32(x.q_smem + kSlot * kTileBytes);
+    const uint32_t k_addr = smem_u32(x.kv_smem + ring.stage * kTileBytes);
+    const uint32_t dS = x.tmem + kSlot * kSlotCols;
+#pragma unroll
+    for (int kk = 0; kk < kD / 16; ++kk) {
+      const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+      umma_ss(dS, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
+              kIdescS, kk > 0);
+    }
+    umma_commit(&sm->s_full[kSlot]);
+    umma_commit(&sm->kv_empty[ring.stage]);
+    if (last) umma_commit(&sm->q_empty[kSlot]);
+  }
+  if (first) ++st.units;
+  st.pend = true;
+  st.pend_j = c.j;
+  ring.next();
+  return true;
+}
+
+// PV event of slot kSlot's pending block (the cursor still points at it).
+// The producer loads V; the MMA thread issues O += P V.
+template <bool kMma, int kSlot>
+__device__ __forceinline__ bool event_pv(SlotState& st, Ring& ring, const Ctx& x) {
+  const Params& p = *x.p;
+  Smem* sm = x.sm;
+  const Cursor& c = st.cur;
+  const bool first = st.pend_j == 0;
+  if (!kMma) {
+    if (!mbar_wait(&sm->kv_empty[ring.stage], ring.phase ^ 1, x.abort)) return false;
+    const int kvbh = (c.bh / p.hq) * p.hkv + (c.bh % p.hq) / p.group;
+    const int vrow = kvbh * p.L + c.list[c.j] * kBlk;
+    uint8_t* dst = x.kv_smem + ring.stage * kTileBytes;
+    mbar_arrive_expect_tx(&sm->kv_full[ring.stage], kTileBytes);
+    tma_load_2d(dst, x.tmV, &sm->kv_full[ring.stage], 0, vrow);
+    tma_load_2d(dst + kHalf, x.tmV, &sm->kv_full[ring.stage], 64, vrow);
+    ++ring.issued;
+  } else {
+    if (!mbar_wait(&sm->p_full[kSlot], st.blocks & 1, x.abort)) return false;
+    // the unit's first PV overwrites O: the previous unit's epilogue must be done
+    if (first && !mbar_wait(&sm->o_empty[kSlot], ((st.units - 1) & 1) ^ 1, x.abort)) return false;
+    if (!mbar_wait(&sm->kv_full[ring.stage], ring.phase, x.abort)) return false;
+    tc_fence_after();
+    const uint32_t v_addr = smem_u32(x.kv_smem + ring.stage * kTileBytes);
+    const uint32_t dO = x.tmem + kSlot * kSlotCols + kColO;
+    const uint32_t aP = x.tmem + kSlot * kSlotCols;
+#pragma unroll
+    for (int kk = 0; kk < kBlk / 16; ++kk) {
+      // 16 keys per step: P columns [8kk, 8kk+8) (bf16 pairs), V rows [16kk, 16kk+16)
+      umma_ts(dO, aP + kk * 8, smem_desc_sw128(v_addr + kk * 16 * 128, kHalf, 1024), kIdescPV,
+              (!first || kk > 0) ? 1u : 0u);
+    }
+    umma_commit(&sm->pv_done[kSlot]);
+    umma_commit(&sm->kv_empty[ring.stage]);
+  }
+  ++st.blocks;
+  st.pend = false;
+  ring.next();
+  return true;
+}
+
+template <bool kMma>
+__device__ __forceinline__ void pipeline(const Params& p, Smem* sm, uint8_t* q_smem,
+                                      uint8_t* kv_smem, uint32_t tmem, const CUtensorMap* tmQ,
+                                      const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                      volatile int* abort) {
+  const Ctx x{&p, sm, q_smem, kv_smem, tmem, tmQ, tmK, tmV, abort};
+  Ring ring{0, 0u, 0};
+  SlotState s0{}, s1{};
+  cursor_init(s0.cur, p, 0);
+  cursor_init(s1.cur, p, 1);
+  bool ok = true;
+  if (s0.cur.valid) ok = event_s<kMma, 0>(s0, ring, x);
+  if (ok && s1.cur.valid) ok = event_s<kMma, 1>(s1, ring, x);
+  while (ok && (s0.pend || s1.pend)) {
+    if (s0.pend) {
+      ok = event_pv<kMma, 0>(s0, ring, x);
+      if (ok && cursor_next(s0.cur, p)) ok = event_s<kMma, 0>(s0, ring, x);
+    }
+    if (ok && s1.pend) {
+      ok = event_pv<kMma, 1>(s1, ring, x);
+      if (ok && cursor_next(s1.cur, p)) ok = event_s<kMma, 1>(s1, ring, x);
+    }
+  }
+  if (!ok && !kMma) {
+    // wait (bounded) for the copies this thread still has in flight
+    const long long nk = ring.issued < kStages ? ring.issued : kStages;
+    for (long long t = 1; t <= nk; ++t) {
+      const long long q = ring.issued - t;
+      const uint32_t addr = smem_u32(&sm->kv_full[q % kStages]);
+      const uint32_t ph = static_cast<uint32_t>((q / kStages) & 1);
+      const unsigned long long t0 = globaltimer();
+      while (!mbar_try_wait(addr, ph) && globaltimer() - t0 < kWaitLimitNs) {
+      }
+    }
+    const uint32_t nu[kSlots] = {s0.units, s1.units};
+    for (int s = 0; s < kSlots; ++s) {
+      if (nu[s] == 0) continue;
+      const uint32_t addr = smem_u32(&sm->q_full[s]);
+      const unsigned long long t0 = globaltimer();
+      while (!mbar_try_wait(addr, (nu[s] - 1) & 1) && globaltimer() - t0 < kWaitLimitNs) {
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* q_smem = base;
-  uint8_t* kv_smem = base + kTileBytes;
-  Smem* sm = reinterpret_cast<Smem*>(base + kTileBytes * (1 + kStages));
+  uint8_t* q_smem = base;                              // kSlots tiles
+  uint8_t* kv_smem = base + kSlots * kTileBytes;       // kStages tiles
+  Smem* sm = reinterpret_cast<Smem*>(base + (kSlots + kStages) * kTileBytes);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
-    mbar_init(&sm->q_full, 1);
-    mbar_init(&sm->q_empty, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm->kv_full[s], 1);
       mbar_init(&sm->kv_empty[s], 1);
     }
-    mbar_init(&sm->s_full, 1);
-    mbar_init(&sm->p_full, 128);
-    mbar_init(&sm->pv_done, 1);
-    mbar_init(&sm->o_empty, 128);
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&sm->q_full[s], 1);
+      mbar_init(&sm->q_empty[s], 1);
+      mbar_init(&sm->s_full[s], 1);
+      mbar_init(&sm->p_full[s], 128);
+      mbar_init(&sm->pv_done[s], 1);
+      mbar_init(&sm->o_empty[s], 128);
+    }
     sm->abort = 0;
     fence_barrier_init();
   }
@@ -114,136 +337,28 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t tmem = sm->tmem_base;
   volatile int* abort = &sm->abort;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------ TMA producer
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t nu = 0;  // units with work seen so far
-      long long issued = 0;
-      bool q_out = false;
-      for (int k = blockIdx.x; k < p.units && !*abort; k += gridDim.x) {
-        const int unit = static_cast<int>(p.order[k]);
-        const int bh = unit / p.NB, qb = unit % p.NB;
-        const int32_t* list = p.idx + static_cast<size_t>(unit) * p.NB;
-        const int n = effective_count(p, list, p.counts[unit], qb);
-        if (n <= 0) continue;
-        const int kvbh = (bh / p.hq) * p.hkv + (bh % p.hq) / p.group;
-        if (!mbar_wait(&sm->q_empty, (nu & 1) ^ 1, abort)) break;
-        mbar_arrive_expect_tx(&sm->q_full, kTileBytes);
-        const int qrow = bh * p.L + qb * kBlk;
-        tma_load_2d(q_smem, &tmQ, &sm->q_full, 0, qrow);
-        tma_load_2d(q_smem + kHalf, &tmQ, &sm->q_full, 64, qrow);
-        q_out = true;
-        for (int j = 0; j < n; ++j) {
-          const int krow = kvbh * p.L + list[j] * kBlk;
-          for (int which = 0; which < 2; ++which) {  // K_j then V_j
-            if (!mbar_wait(&sm->kv_empty[stage], phase ^ 1, abort)) goto producer_done;
-            uint8_t* dst = kv_smem + stage * kTileBytes;
-            const CUtensorMap* map = which == 0 ? &tmK : &tmV;
-            mbar_arrive_expect_tx(&sm->kv_full[stage], kTileBytes);
-            tma_load_2d(dst, map, &sm->kv_full[stage], 0, krow);
-            tma_load_2d(dst + kHalf, map, &sm->kv_full[stage], 64, krow);
-            ++issued;
-            if (++stage == kStages) {
-              stage = 0;
-              phase ^= 1;
-            }
-          }
-        }
-        ++nu;
-      }
-    producer_done:
-      if (*abort) {
-        // wait (bounded) for the copies this thread still has in flight
-        const long long nk = issued < kStages ? issued : kStages;
-        for (long long t = 1; t <= nk; ++t) {
-          const long long q = issued - t;
-          const uint32_t addr = smem_u32(&sm->kv_full[q % kStages]);
-          const uint32_t ph = static_cast<uint32_t>((q / kStages) & 1);
-          const unsigned long long t0 = globaltimer();
-          while (!mbar_try_wait(addr, ph) && globaltimer() - t0 < kWaitLimitNs) {
-          }
-        }
-        if (q_out && nu > 0) {
-          const uint32_t addr = smem_u32(&sm->q_full);
-          const unsigned long long t0 = globaltimer();
-          while (!mbar_try_wait(addr, (nu - 1) & 1) && globaltimer() - t0 < kWaitLimitNs) {
-          }
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------ MMA issuer
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t nu = 0;
-      uint32_t g = 0;  // global block counter of this CTA
-      const uint32_t q_addr = smem_u32(q_smem);
-      for (int k = blockIdx.x; k < p.units; k += gridDim.x) {
-        const int unit = static_cast<int>(p.order[k]);
-        const int qb = unit % p.NB;
-        const int32_t* list = p.idx + static_cast<size_t>(unit) * p.NB;
-        const int n = effective_count(p, list, p.counts[unit], qb);
-        if (n <= 0) continue;
-        if (!mbar_wait(&sm->q_full, nu & 1, abort)) goto mma_done;
-        for (int j = 0; j < n; ++j, ++g) {
-          // S_j = Q K_j^T
-          if (!mbar_wait(&sm->kv_full[stage], phase, abort)) goto mma_done;
-          tc_fence_after();
-          {
-            const uint32_t k_addr = smem_u32(kv_smem + stage * kTileBytes);
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-              umma_ss(tmem + kColS, smem_desc_sw128(q_addr + off, 16, 1024),
-                      smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0);
-            }
-          }
-          umma_commit(&sm->s_full);
-          umma_commit(&sm->kv_empty[stage]);
-          if (j == n - 1) umma_commit(&sm->q_empty);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
-          // O += P_j V_j
-          if (!mbar_wait(&sm->p_full, g & 1, abort)) goto mma_done;
-          if (j == 0 && !mbar_wait(&sm->o_empty, (nu & 1) ^ 1, abort)) goto mma_done;
-          if (!mbar_wait(&sm->kv_full[stage], phase, abort)) goto mma_done;
-          tc_fence_after();
-          {
-            const uint32_t v_addr = smem_u32(kv_smem + stage * kTileBytes);
-#pragma unroll
-            for (int kk = 0; kk < kBlk / 16; ++kk) {
-              // 16 keys per step: P columns [8kk, 8kk+8) (bf16 pairs), V rows [16kk, 16kk+16)
-              umma_ts(tmem + kColO, tmem + kColS + kk * 8,
-                      smem_desc_sw128(v_addr + kk * 16 * 128, kHalf, 1024), kIdescPV,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-            }
-          }
-          umma_commit(&sm->pv_done);
-          umma_commit(&sm->kv_empty[stage]);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-        ++nu;
-      }
-    mma_done:;
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");  // 128 x 80
+    if (warp <= 1 && lane == 0) {
+      // Producer (warp 0) and MMA issuer (warp 1) walk the same merged event
+      // order: S(0), S(1), { PV(0), S(0, next), PV(1), S(1, next) } ...
+      if (warp == 0)
+        pipeline<false>(p, sm, q_smem, kv_smem, tmem, &tmQ, &tmK, &tmV, abort);
+      else
+        pipeline<true>(p, sm, q_smem, kv_smem, tmem, &tmQ, &tmK, &tmV, abort);
     }
   } else {
     // ------------------------------------------------ softmax + epilogue
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n" ::: "memory");  // 256 x 208
+    const int slot = (warp - 4) / 4;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_addr + kColS;
-    const uint32_t tO = tmem + lane_addr + kColO;
+    const uint32_t tS = tmem + lane_addr + slot * kSlotCols;
+    const uint32_t tO = tS + kColO;
     const float sl2 = p.scale_log2;
-    uint32_t g = 0;
-    for (int k = blockIdx.x; k < p.units; k += gridDim.x) {
+    uint32_t g = 0;  // blocks processed by this slot
+    for (int k = 2 * blockIdx.x + slot; k < p.units; k += 2 * gridDim.x) {
       const int unit = static_cast<int>(p.order[k]);
       const int bh = unit / p.NB, qb = unit % p.NB;
       const int32_t* list = p.idx + static_cast<size_t>(unit) * p.NB;
@@ -251,88 +366,98 @@ __global__ void __launch_bounds__(kThreads, 2)
       const size_t orow = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qb) * kBlk + row;
       __nv_bfloat16* optr = p.O + orow * kD;
       if (n <= 0) {
-        uint4 z = make_uint4(0, 0, 0, 0);
+        const uint4 z = make_uint4(0, 0, 0, 0);
         for (int c = 0; c < kD / 8; ++c) reinterpret_cast<uint4*>(optr)[c] = z;
         if (p.lse) p.lse[orow] = -INFINITY;
         continue;
       }
+      // a causal list is ascending and ends at most at qb: only its last
+      // block can be the diagonal one
+      const bool last_is_diag = p.causal && list[n - 1] == qb;
       float m_run = -INFINITY;  // running max of scaled logits (log2 units)
       float l_run = 0.f;
       bool failed = false;
       for (int j = 0; j < n; ++j, ++g) {
-        const bool diag = p.causal && list[j] == qb;
-        if (!warp_wait(&sm->s_full, g & 1, abort)) {
+        const bool diag = last_is_diag && j == n - 1;
+        if (!warp_wait(&sm->s_full[slot], g & 1, abort)) {
           failed = true;
           break;
         }
         tc_fence_after();
-        float s[kBlk];
+        uint32_t sv[4][32];
 #pragma unroll
-        for (int c = 0; c < kBlk / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tS + c * 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(v[i]);
-        }
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sv[c]);
+        tmem_ld_wait();
+        float mx = -INFINITY;
         if (diag) {
 #pragma unroll
-          for (int c = 0; c < kBlk; ++c)
-            if (c > row) s[c] = -INFINITY;
-        }
-        float mx = -INFINITY;
+          for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int c = 0; c < kBlk; ++c) mx = fmaxf(mx, s[c]);
+            for (int i = 0; i < 32; ++i)
+              if (c * 32 + i > row) sv[c][i] = __float_as_uint(-INFINITY);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sv[c][i]));
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool need = m_new > m_run + kRescaleLog2;
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? ex2(m_run - m_new) : 1.0f;
-          if (j > 0) {
-            // O holds PV_0..PV_{j-1}: wait for the last one, then rescale in place
-            if (!warp_wait(&sm->pv_done, (g - 1) & 1, abort)) {
-              failed = true;
-              break;
-            }
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < kD / 32; ++c) {
-              uint32_t v[32];
-              tmem_ld32(tO + c * 32, v);
-              tmem_ld_wait();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-              tmem_st32(tO + c * 32, v);
-            }
-            tmem_st_wait();
-          }
-          if (need) {
-            l_run *= alpha;
-            m_run = m_new;
-          }
+        const bool any_need = __any_sync(0xffffffffu, need);
+        const float alpha = need ? ex2(m_run - m_new) : 1.0f;
+        if (need) {
+          l_run *= alpha;
+          m_run = m_new;
         }
-        const float mb = m_run;
-        float lsum = 0.f;
+        const unsigned long long scale2 = f2_pack(sl2, sl2);
+        const unsigned long long negm2 = f2_pack(-m_run, -m_run);
+        unsigned long long lsum2 = f2_pack(0.f, 0.f);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           // keys [64h, 64h + 64) -> bf16 pairs in TMEM columns [32h, 32h + 32)
           uint32_t pk[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2(fmaf(s[64 * h + 2 * c], sl2, -mb));
-            const float p1 = ex2(fmaf(s[64 * h + 2 * c + 1], sl2, -mb));
-            lsum += p0 + p1;
+            const int e = 64 * h + 2 * c;
+            const unsigned long long x2 =
+                f2_pack(__uint_as_float(sv[e >> 5][e & 31]),
+                        __uint_as_float(sv[(e + 1) >> 5][(e + 1) & 31]));
+            float a0, a1;
+            f2_unpack(f2_fma(x2, scale2, negm2), a0, a1);
+            const float p0 = ex2(a0);
+            const float p1 = ex2(a1);
+            lsum2 = f2_add(lsum2, f2_pack(p0, p1));
             pk[c] = pack_bf16x2(p0, p1);
           }
           tmem_st32(tS + 32 * h, pk);
         }
-        l_run += lsum;
+        float ls0, ls1;
+        f2_unpack(lsum2, ls0, ls1);
+        l_run += ls0 + ls1;
+        if (any_need && j > 0) {
+          // O holds PV_0..PV_{j-1}: wait for the last one, then rescale in place
+          // (PV_j cannot start before this thread arrives on p_full below)
+          if (!warp_wait(&sm->pv_done[slot], (g - 1) & 1, abort)) {
+            failed = true;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < kD / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tO + c * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+            tmem_st32(tO + c * 32, v);
+          }
+        }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&sm->p_full);
+        mbar_arrive(&sm->p_full[slot]);
       }
       if (failed) break;
       // ---- epilogue: O / l -> bf16 rows
-      if (!warp_wait(&sm->pv_done, (g - 1) & 1, abort)) break;
+      if (!warp_wait(&sm->pv_done[slot], (g - 1) & 1, abort)) break;
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;
 #pragma unroll 1
@@ -350,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       if (p.lse) p.lse[orow] = (m_run + lg2(l_run)) * 0.69314718055994531f;
       tc_fence_before();
-      mbar_arrive(&sm->o_empty);
+      mbar_arrive(&sm->o_empty[slot]);
     }
   }
 
@@ -382,12 +507,13 @@ cudaError_t launch_attn_tc(const Dims& D, const CUtensorMap& tmQ, const CUtensor
   p.O = static_cast<__nv_bfloat16*>(O);
   p.lse = lse;
   p.status = status;
-  const size_t smem = 1024 + kTileBytes * (1 + kStages) + sizeof(Smem);
+  const size_t smem = 1024 + kTileBytes * (kSlots + kStages) + sizeof(Smem);
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  int grid = 2 * num_sms;
-  if (grid > p.units) grid = p.units;
+  int grid = num_sms;
+  const int need = (p.units + 1) / 2;
+  if (grid > need) grid = need;
   if (grid < 1) grid = 1;
   attn_tc_kernel<<<grid, kThreads, smem, st>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();

@@ -19,7 +19,9 @@ constexpr int kThreads = 256;
 __global__ void __launch_bounds__(kThreads)
     score_reduce_kernel(const float* __restrict__ part, float* __restrict__ probs, int NB, int r,
                         int R, int causal) {
-  extern __shared__ float lse[];  // r entries
+  extern __shared__ float smem[];
+  float* lse = smem;                                   // r entries
+  size_t* row_off = reinterpret_cast<size_t*>(smem + ((r + 1) & ~1));  // r entries
   const int b = blockIdx.x;
   const int bh = blockIdx.y;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -27,29 +29,62 @@ __global__ void __launch_bounds__(kThreads)
   const int nj = causal ? b + 1 : NB;
   const float* base = part + static_cast<size_t>(bh) * part_head_elems(NB, r, R, causal != 0);
 
+  for (int t = threadIdx.x; t < r; t += kThreads)
+    row_off[t] = part_row_offset(b * r + t, r, NB, causal != 0);
+  __syncthreads();
+  // row log-sum-exp: online (max, sum) over 8 loads in flight per lane
   for (int t = warp; t < r; t += nwarps) {
-    const float* row = base + part_row_offset(b * r + t, r, NB, causal != 0);
-    float m = -INFINITY;
-    for (int j = lane; j < nj; j += 32) m = fmaxf(m, row[j]);
+    const float* row = base + row_off[t];
+    float m = -INFINITY, s = 0.f;
+    for (int j0 = 0; j0 < nj; j0 += 8 * 32) {
+      float v[8];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float s = 0.f;
-    for (int j = lane; j < nj; j += 32) s += ex2(row[j] - m);
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * 32 + lane;
+        v[u] = j < nj ? __ldg(row + j) : -INFINITY;
+      }
+      float cm = m;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      for (int u = 0; u < 8; ++u) cm = fmaxf(cm, v[u]);
+      if (cm != -INFINITY) {
+        float cs = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) cs += ex2(v[u] - cm);
+        s = s * ex2(m - cm) + cs;
+        m = cm;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+      const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+      const float mm = fmaxf(m, m2);
+      if (mm != -INFINITY) {
+        s = s * ex2(m - mm) + s2 * ex2(m2 - mm);
+        m = mm;
+      }
+    }
     if (lane == 0) lse[t] = m + lg2(s);
   }
   __syncthreads();
 
+  // P[b, j] = (1/r) sum_t 2^(part[t][j] - lse[t]); r loads in flight per thread
   float* out = probs + (static_cast<size_t>(bh) * NB + b) * NB;
   const float inv_r = 1.0f / static_cast<float>(r);
   for (int j = threadIdx.x; j < NB; j += kThreads) {
     float acc = 0.f;
     if (j < nj) {
-      for (int t = 0; t < r; ++t) {
-        const float* row = base + part_row_offset(b * r + t, r, NB, causal != 0);
-        acc += ex2(row[j] - lse[t]);
+      int t = 0;
+      for (; t + 8 <= r; t += 8) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          v[u] = __ldg(base + row_off[t + u] + j);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc += ex2(v[u] - lse[t + u]);
       }
+      for (; t < r; ++t)
+        acc += ex2(__ldg(base + row_off[t] + j) - lse[t]);
     }
     out[j] = acc * inv_r;
   }
@@ -60,8 +95,8 @@ __global__ void __launch_bounds__(kThreads)
 cudaError_t launch_score_reduce(const Dims& D, const float* part, float* probs,
                                 cudaStream_t st) {
   dim3 grid(D.NB, D.batch * D.hq);
-  score_reduce_kernel<<<grid, kThreads, D.r * sizeof(float), st>>>(part, probs, D.NB, D.r, D.R,
-                                                                   D.causal);
+  const size_t smem = ((D.r + 1) & ~1) * sizeof(float) + D.r * sizeof(size_t);
+  score_reduce_kernel<<<grid, kThreads, smem, st>>>(part, probs, D.NB, D.r, D.R, D.causal);
   return cudaGetLastError();
 }
 

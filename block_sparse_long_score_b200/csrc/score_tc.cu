@@ -57,6 +57,16 @@ struct Smem {
   int abort;
 };
 
+// Number of causal tiles in tile rows [0, m): sum over rows of min(NT, row/2 + 1).
+// Rows below 2*NT are uncapped: sum_{i<m} (floor(i/2) + 1) = m + q(q-1) (m = 2q)
+// or m + q^2 (m = 2q + 1).
+__host__ __device__ __forceinline__ long long tiles_before(int m, int NT) {
+  const long long mu = m < 2 * NT ? m : 2 * NT;
+  const long long q = mu >> 1;
+  const long long uncapped = mu + ((mu & 1) ? q * q : q * (q - 1));
+  return uncapped + static_cast<long long>(NT) * (m > 2 * NT ? m - 2 * NT : 0);
+}
+
 __device__ __forceinline__ void decode_tile(long long t, const Params& p, int& bh, int& mt,
                                             int& nt) {
   bh = static_cast<int>(t / p.tiles_per_head);
@@ -66,17 +76,16 @@ __device__ __forceinline__ void decode_tile(long long t, const Params& p, int& b
     nt = rem % p.NT;
     return;
   }
-  // Causal: tile row mt needs key tiles nt with nt*256 <= mt*128 + 127,
-  // i.e. nt <= mt / 2.
-  int m = 0;
-  for (;;) {
-    const int c = min(p.NT, (m >> 1) + 1);
-    if (rem < c) break;
-    rem -= c;
-    ++m;
+  // Causal: tile row m needs key tiles nt with nt*256 <= m*128 + 127, i.e.
+  // nt <= m / 2, so it holds min(NT, m/2 + 1) tiles. Bisection on the
+  // closed-form count of tiles in rows [0, m).
+  int lo = 0, hi = p.MT;  // invariant: tiles_before(lo) <= rem < tiles_before(hi)
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (tiles_before(mid, p.NT) <= rem) lo = mid; else hi = mid;
   }
-  mt = m;
-  nt = rem;
+  mt = lo;
+  nt = rem - static_cast<int>(tiles_before(lo, p.NT));
 }
 
 // Reduces one 32-column chunk of a row into per-key-block partials.
@@ -337,6 +346,7 @@ cudaError_t launch_score_tc(const Dims& D, const CUtensorMap& tmQ, const CUtenso
   if (D.causal) {
     long long n = 0;
     for (int m = 0; m < p.MT; ++m) n += (m / 2 + 1 < p.NT) ? (m / 2 + 1) : p.NT;
+    if (n != tiles_before(p.MT, p.NT)) return cudaErrorInvalidValue;  // closed form check
     p.tiles_per_head = static_cast<int>(n);
   } else {
     p.tiles_per_head = p.MT * p.NT;

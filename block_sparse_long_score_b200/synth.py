@@ -35,7 +35,7 @@ __all__ = ["Problem", "CONFIGS", "make_problem", "SLASH_GAMMA"]
 # Amplitude of the slash-band process (a free constant of the recipe). It is
 # picked once, on the 256K Llama-shaped layer, to give a block density near the
 # ~7 % that the paper reports at 256K. The same value is used at every length.
-SLASH_GAMMA = 0.60
+SLASH_GAMMA = 0.755
 
 
 @dataclass
