@@ -396,10 +396,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i)
               if (c * 32 + i > row) sv[c][i] = __float_as_uint(-INFINITY);
         }
+        {
+          // 8 independent partial maxima: a short dependency chain
+          float pm[8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+          for (int q = 0; q < 8; ++q) pm[q] = __uint_as_float(sv[q >> 1][(q & 1) * 16]);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sv[c][i]));
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int q = c * 2 + (i >> 4);
+              if ((i & 15) != 0) pm[q] = fmaxf(pm[q], __uint_as_float(sv[c][i]));
+            }
+          mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                     fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        }
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool need = m_new > m_run + kRescaleLog2;
         const bool any_need = __any_sync(0xffffffffu, need);
@@ -410,7 +421,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const unsigned long long scale2 = f2_pack(sl2, sl2);
         const unsigned long long negm2 = f2_pack(-m_run, -m_run);
-        unsigned long long lsum2 = f2_pack(0.f, 0.f);
+        unsigned long long lsum2[4];   // 4 independent pair-accumulators
+#pragma unroll
+        for (int q = 0; q < 4; ++q) lsum2[q] = f2_pack(0.f, 0.f);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           // keys [64h, 64h + 64) -> bf16 pairs in TMEM columns [32h, 32h + 32)
@@ -425,14 +438,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             f2_unpack(f2_fma(x2, scale2, negm2), a0, a1);
             const float p0 = ex2(a0);
             const float p1 = ex2(a1);
-            lsum2 = f2_add(lsum2, f2_pack(p0, p1));
+            lsum2[c & 3] = f2_add(lsum2[c & 3], f2_pack(p0, p1));
             pk[c] = pack_bf16x2(p0, p1);
           }
           tmem_st32(tS + 32 * h, pk);
         }
-        float ls0, ls1;
-        f2_unpack(lsum2, ls0, ls1);
-        l_run += ls0 + ls1;
+        float ls0, ls1, ls2, ls3, ls4, ls5, ls6, ls7;
+        f2_unpack(lsum2[0], ls0, ls1);
+        f2_unpack(lsum2[1], ls2, ls3);
+        f2_unpack(lsum2[2], ls4, ls5);
+        f2_unpack(lsum2[3], ls6, ls7);
+        l_run += ((ls0 + ls1) + (ls2 + ls3)) + ((ls4 + ls5) + (ls6 + ls7));
         if (any_need && j > 0) {
           // O holds PV_0..PV_{j-1}: wait for the last one, then rescale in place
           // (PV_j cannot start before this thread arrives on p_full below)
