@@ -191,7 +191,7 @@ int xattn_select(const float* probs, const float* tau, const xattn_shape* shape,
 size_t xattn_attn_workspace_bytes(const xattn_shape* shape) {
   Dims D;
   if (check_shape(shape, &D) != XATTN_OK) return 0;
-  return sizeof(uint32_t) * (static_cast<size_t>(D.batch) * D.hq * D.NB + 64);
+  return sizeof(unsigned long long) * (static_cast<size_t>(D.batch) * D.hq * D.NB + 32);
 }
 
 int xattn_sparse_attn(const void* Q, const void* K, const void* V, const xattn_shape* shape,
@@ -209,8 +209,8 @@ int xattn_sparse_attn(const void* Q, const void* K, const void* V, const xattn_s
   if ((rc = device_state(&ds)) != XATTN_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (D.dtype == XATTN_BF16) {
-    uint32_t* order = static_cast<uint32_t*>(ws);
-    if ((rc = cuda_status(launch_sched(D, counts, order, st))) != XATTN_OK) return rc;
+    unsigned long long* order = static_cast<unsigned long long*>(ws);
+    if ((rc = cuda_status(launch_sched(D, counts, idx, order, st))) != XATTN_OK) return rc;
     CUtensorMap tq, tk, tv;
     if ((rc = make_map_2d(&tq, Q, static_cast<long long>(D.batch) * D.hq * D.L)) != XATTN_OK)
       return rc;

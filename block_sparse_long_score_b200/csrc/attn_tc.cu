@@ -63,7 +63,7 @@ struct Params {
   float scale_log2;  // log2(e) / sqrt(d)
   const int32_t* counts;
   const int32_t* idx;
-  const uint32_t* order;
+  const unsigned long long* order;  // packed entries: unit | n << 32 | diag << 48
   __nv_bfloat16* O;
   float* lse;
   int* status;
@@ -77,53 +77,83 @@ struct Smem {
   int abort;
 };
 
+// One packed work-order entry (written by the schedule kernel).
+constexpr unsigned long long kEndEntry = ~0ull;
+
+__device__ __forceinline__ unsigned long long load_entry(const Params& p, int k) {
+  return k < p.units ? __ldg(p.order + k) : kEndEntry;
+}
+__device__ __forceinline__ int entry_unit(unsigned long long e) {
+  return static_cast<int>(e & 0xFFFFFFFFull);
+}
+__device__ __forceinline__ int entry_count(unsigned long long e) {
+  return static_cast<int>((e >> 32) & 0xFFFFull);
+}
+__device__ __forceinline__ bool entry_diag(unsigned long long e) { return (e >> 48) & 1ull; }
+
 // Walks the blocks of one slot's units in order, skipping units with no block.
+// The next unit's entry is always one load ahead; the producer (kList) also
+// keeps the next block index of the list one load ahead.
 struct Cursor {
   int k;        // position in the unit order
   int step;     // distance between this slot's units (2 * grid)
   int unit, bh, qb, n, j;
   const int32_t* list;
+  int kb, kb_next;                // list[j], list[j + 1]
+  unsigned long long next_entry;  // order entry at position k (before a seek)
   bool valid;
 };
 
-__device__ __forceinline__ int effective_count(const Params& p, const int32_t* list, int n,
-                                               int qb) {
-  n = n < 0 ? 0 : (n > p.NB ? p.NB : n);
-  if (!p.causal) return n;
-  while (n > 0 && list[n - 1] > qb) --n;  // ascending list: drop blocks above the diagonal
-  return n;
-}
-
+template <bool kList>
 __device__ __forceinline__ void cursor_seek(Cursor& c, const Params& p) {
-  for (; c.k < p.units; c.k += c.step) {
-    c.unit = static_cast<int>(p.order[c.k]);
-    c.bh = c.unit / p.NB;
-    c.qb = c.unit % p.NB;
-    c.list = p.idx + static_cast<size_t>(c.unit) * p.NB;
-    c.n = effective_count(p, c.list, p.counts[c.unit], c.qb);
-    c.j = 0;
-    if (c.n > 0) {
+  for (;;) {
+    if (c.k >= p.units) {
+      c.valid = false;
+      return;
+    }
+    const unsigned long long e = c.next_entry;
+    c.next_entry = load_entry(p, c.k + c.step);  // prefetch the following unit
+    const int n = entry_count(e);
+    if (n > 0) {
+      c.unit = entry_unit(e);
+      c.bh = c.unit / p.NB;
+      c.qb = c.unit % p.NB;
+      c.list = p.idx + static_cast<size_t>(c.unit) * p.NB;
+      c.n = n;
+      c.j = 0;
+      if (kList) {
+        c.kb = c.list[0];
+        c.kb_next = n > 1 ? c.list[1] : 0;
+      }
       c.valid = true;
       return;
     }
+    c.k += c.step;
   }
-  c.valid = false;
 }
 
+template <bool kList>
 __device__ __forceinline__ void cursor_init(Cursor& c, const Params& p, int slot) {
   c.k = 2 * blockIdx.x + slot;
   c.step = 2 * gridDim.x;
-  cursor_seek(c, p);
+  c.next_entry = load_entry(p, c.k);
+  cursor_seek<kList>(c, p);
 }
 
 // Moves past the current block; returns false when the slot has no more work.
+template <bool kList>
 __device__ __forceinline__ bool cursor_next(Cursor& c, const Params& p) {
-  if (++c.j < c.n) return true;
+  if (++c.j < c.n) {
+    if (kList) {
+      c.kb = c.kb_next;
+      if (c.j + 1 < c.n) c.kb_next = c.list[c.j + 1];
+    }
+    return true;
+  }
   c.k += c.step;
-  cursor_seek(c, p);
+  cursor_seek<kList>(c, p);
   return c.valid;
 }
-
 
 struct SlotState {
   Cursor cur;
@@ -176,7 +206,7 @@ __device__ __forceinline__ bool event_s(SlotState& st, Ring& ring, const Ctx& x)
     }
     if (!mbar_wait(&sm->kv_empty[ring.stage], ring.phase ^ 1, x.abort)) return false;
     const int kvbh = (c.bh / p.hq) * p.hkv + (c.bh % p.hq) / p.group;
-    const int krow = kvbh * p.L + c.list[c.j] * kBlk;
+    const int krow = kvbh * p.L + c.kb * kBlk;
     uint8_t* dst = x.kv_smem + ring.stage * kTileBytes;
     mbar_arrive_expect_tx(&sm->kv_full[ring.stage], kTileBytes);
     tma_load_2d(dst, x.tmK, &sm->kv_full[ring.stage], 0, krow);
@@ -217,7 +247,7 @@ __device__ __forceinline__ bool event_pv(SlotState& st, Ring& ring, const Ctx& x
   if (!kMma) {
     if (!mbar_wait(&sm->kv_empty[ring.stage], ring.phase ^ 1, x.abort)) return false;
     const int kvbh = (c.bh / p.hq) * p.hkv + (c.bh % p.hq) / p.group;
-    const int vrow = kvbh * p.L + c.list[c.j] * kBlk;
+    const int vrow = kvbh * p.L + c.kb * kBlk;
     uint8_t* dst = x.kv_smem + ring.stage * kTileBytes;
     mbar_arrive_expect_tx(&sm->kv_full[ring.stage], kTileBytes);
     tma_load_2d(dst, x.tmV, &sm->kv_full[ring.stage], 0, vrow);
@@ -255,19 +285,19 @@ __device__ __forceinline__ void pipeline(const Params& p, Smem* sm, uint8_t* q_s
   const Ctx x{&p, sm, q_smem, kv_smem, tmem, tmQ, tmK, tmV, abort};
   Ring ring{0, 0u, 0};
   SlotState s0{}, s1{};
-  cursor_init(s0.cur, p, 0);
-  cursor_init(s1.cur, p, 1);
+  cursor_init<!kMma>(s0.cur, p, 0);
+  cursor_init<!kMma>(s1.cur, p, 1);
   bool ok = true;
   if (s0.cur.valid) ok = event_s<kMma, 0>(s0, ring, x);
   if (ok && s1.cur.valid) ok = event_s<kMma, 1>(s1, ring, x);
   while (ok && (s0.pend || s1.pend)) {
     if (s0.pend) {
       ok = event_pv<kMma, 0>(s0, ring, x);
-      if (ok && cursor_next(s0.cur, p)) ok = event_s<kMma, 0>(s0, ring, x);
+      if (ok && cursor_next<!kMma>(s0.cur, p)) ok = event_s<kMma, 0>(s0, ring, x);
     }
     if (ok && s1.pend) {
       ok = event_pv<kMma, 1>(s1, ring, x);
-      if (ok && cursor_next(s1.cur, p)) ok = event_s<kMma, 1>(s1, ring, x);
+      if (ok && cursor_next<!kMma>(s1.cur, p)) ok = event_s<kMma, 1>(s1, ring, x);
     }
   }
   if (!ok && !kMma) {
@@ -358,11 +388,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tS + kColO;
     const float sl2 = p.scale_log2;
     uint32_t g = 0;  // blocks processed by this slot
+    unsigned long long e_next = load_entry(p, 2 * blockIdx.x + slot);
     for (int k = 2 * blockIdx.x + slot; k < p.units; k += 2 * gridDim.x) {
-      const int unit = static_cast<int>(p.order[k]);
+      const unsigned long long e = e_next;
+      e_next = load_entry(p, k + 2 * gridDim.x);  // prefetch the next unit's entry
+      const int unit = entry_unit(e);
       const int bh = unit / p.NB, qb = unit % p.NB;
-      const int32_t* list = p.idx + static_cast<size_t>(unit) * p.NB;
-      const int n = effective_count(p, list, p.counts[unit], qb);
+      const int n = entry_count(e);
       const size_t orow = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qb) * kBlk + row;
       __nv_bfloat16* optr = p.O + orow * kD;
       if (n <= 0) {
@@ -372,8 +404,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       // a causal list is ascending and ends at most at qb: only its last
-      // block can be the diagonal one
-      const bool last_is_diag = p.causal && list[n - 1] == qb;
+      // block can be the diagonal one (flagged in the order entry)
+      const bool last_is_diag = entry_diag(e);
       float m_run = -INFINITY;  // running max of scaled logits (log2 units)
       float l_run = 0.f;
       bool failed = false;
@@ -506,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_attn_tc(const Dims& D, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                            const CUtensorMap& tmV, const int32_t* counts, const int32_t* idx,
-                           const uint32_t* order, void* O, float* lse, int* status,
+                           const unsigned long long* order, void* O, float* lse, int* status,
                            int num_sms, cudaStream_t st) {
   Params p{};
   p.L = D.L;

@@ -61,14 +61,15 @@ struct TauArg {
 cudaError_t launch_select(const Dims& D, const float* probs, const TauArg& tau, uint32_t* mask,
                           int32_t* counts, int32_t* idx, cudaStream_t st);
 
-// Longest-list-first order of the work units (bh, b) into `order`.
-cudaError_t launch_sched(const Dims& D, const int32_t* counts, uint32_t* order,
-                         cudaStream_t st);
+// Longest-list-first order of the work units (bh, b) into `order`: one packed
+// 64-bit entry per unit (unit index, effective block count, diagonal flag).
+cudaError_t launch_sched(const Dims& D, const int32_t* counts, const int32_t* idx,
+                         unsigned long long* order, cudaStream_t st);
 
 // bf16 tensor-core block-sparse attention.
 cudaError_t launch_attn_tc(const Dims& D, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                            const CUtensorMap& tmV, const int32_t* counts, const int32_t* idx,
-                           const uint32_t* order, void* O, float* lse, int* status,
+                           const unsigned long long* order, void* O, float* lse, int* status,
                            int num_sms, cudaStream_t st);
 
 // fp32 CUDA-core block-sparse attention.

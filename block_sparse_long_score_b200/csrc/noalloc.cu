@@ -1,14 +1,14 @@
 // noalloc.cu -- xattn_sparse_attn_noalloc: block-sparse attention for callers
 // that cannot allocate device memory.
 //
-// xattn_sparse_attn needs a small workspace for its work order (one uint32
-// per work unit). Some callers have no way to provide it: a host program that
+// xattn_sparse_attn needs a small workspace for its work order (one 64-bit
+// entry per work unit). Some callers have no way to provide it: a host program that
 // has handed all device memory to another allocator, or a serving loop that may
 // not allocate once it is running (cudaMalloc can synchronise the device and
 // can fail under memory pressure). This entry point keeps that order list in a
 // file-scope __device__ array instead, so it allocates nothing.
 //
-// The array holds XATTN_NOALLOC_MAX_UNITS entries (1 MiB). Every GPU that loads
+// The array holds XATTN_NOALLOC_MAX_UNITS entries (2 MiB). Every GPU that loads
 // the library keeps it until the process exits. All calls on a device share it
 // and it keeps the last call's contents; the schedule kernel rewrites every
 // entry a call reads, so nothing needs clearing. Calls whose kernels overlap on
@@ -24,15 +24,15 @@ namespace xattn {
 namespace {
 
 // Work-order scratch of xattn_sparse_attn_noalloc (device memory of the module).
-static __device__ __align__(256) uint32_t g_noalloc_order[XATTN_NOALLOC_MAX_UNITS];
+static __device__ __align__(256) unsigned long long g_noalloc_order[XATTN_NOALLOC_MAX_UNITS];
 
 std::mutex g_scratch_mu;
-uint32_t* g_scratch_ptr[host::kMaxDevices] = {};
+unsigned long long* g_scratch_ptr[host::kMaxDevices] = {};
 
 // Device address of g_noalloc_order on the current device. In host code the
 // symbol itself is only a host-side stand-in, so the address is looked up
 // once per device with cudaGetSymbolAddress and cached.
-int scratch_address(uint32_t** out) {
+int scratch_address(unsigned long long** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= host::kMaxDevices)
     return XATTN_ERR_CUDA;
@@ -41,7 +41,7 @@ int scratch_address(uint32_t** out) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_order) != cudaSuccess || p == nullptr)
       return XATTN_ERR_CUDA;
-    g_scratch_ptr[dev] = static_cast<uint32_t*>(p);
+    g_scratch_ptr[dev] = static_cast<unsigned long long*>(p);
   }
   *out = g_scratch_ptr[dev];
   return XATTN_OK;
@@ -75,9 +75,9 @@ extern "C" int xattn_sparse_attn_noalloc(const void* Q, const void* K, const voi
     return XATTN_ERR_INVALID_ARG;
   DeviceState* ds = nullptr;
   if ((rc = device_state(&ds)) != XATTN_OK) return rc;
-  uint32_t* order = nullptr;
+  unsigned long long* order = nullptr;
   if ((rc = scratch_address(&order)) != XATTN_OK) return rc;
-  if ((rc = cuda_status(launch_sched(D, counts, order, st))) != XATTN_OK) return rc;
+  if ((rc = cuda_status(launch_sched(D, counts, idx, order, st))) != XATTN_OK) return rc;
   CUtensorMap tq, tk, tv;
   if ((rc = make_map_2d(&tq, Q, static_cast<long long>(D.batch) * D.hq * D.L)) != XATTN_OK)
     return rc;

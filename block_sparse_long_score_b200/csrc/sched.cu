@@ -2,9 +2,16 @@
 //
 // A work unit is one (batch*head, query block) pair; its cost is proportional
 // to its number of selected key blocks. Causal lists grow with the query-block
-// index, so the units are ordered by count, descending (a counting sort over
-// counts 0..NB in one CTA). The persistent attention CTAs then take units
+// index, so the units are ordered by block count, descending (a counting sort
+// over counts 0..NB in one CTA). The persistent attention CTAs take units
 // round-robin from this order, which spreads the long lists first.
+//
+// Each order entry packs everything the attention kernel needs to start a
+// unit into one 64-bit word, so that it costs one (prefetchable) load:
+//   bits  0..31  unit index (bh * NB + query block)
+//   bits 32..47  effective block count: causal lists drop trailing blocks above
+//                the diagonal (lists are ascending)
+//   bit  48      the last listed block is the diagonal block (causal)
 #include "common.cuh"
 
 namespace xattn {
@@ -12,17 +19,59 @@ namespace {
 
 constexpr int kThreads = 1024;
 
+// Effective block count and diagonal flag of units u, u + kThreads, ...
+// (8 of them): causal lists drop trailing blocks above the diagonal.
+__device__ __forceinline__ void unit_info8(const int32_t* __restrict__ counts,
+                                           const int32_t* __restrict__ idx, int u, int units,
+                                           int NB, int causal, int (&n)[8], bool (&diag)[8]) {
+  int c[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int uu = u + q * kThreads;
+    const int v = uu < units ? counts[uu] : 0;
+    c[q] = v < 0 ? 0 : (v > NB ? NB : v);
+  }
+  if (causal) {
+    int last[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int uu = u + q * kThreads;
+      last[q] = (uu < units && c[q] > 0) ? idx[static_cast<size_t>(uu) * NB + c[q] - 1] : -1;
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int uu = u + q * kThreads;
+      const int qb = uu % NB;
+      if (uu < units && last[q] > qb) {  // rare: trailing blocks above the diagonal
+        const int32_t* list = idx + static_cast<size_t>(uu) * NB;
+        while (c[q] > 0 && list[c[q] - 1] > qb) --c[q];
+        last[q] = c[q] > 0 ? list[c[q] - 1] : -1;
+      }
+      diag[q] = uu < units && c[q] > 0 && last[q] == qb;
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) diag[q] = false;
+  }
+#pragma unroll
+  for (int q = 0; q < 8; ++q) n[q] = c[q];
+}
+
 __global__ void __launch_bounds__(kThreads)
-    sched_kernel(const int32_t* __restrict__ counts, int units, int NB,
-                 uint32_t* __restrict__ order) {
+    sched_kernel(const int32_t* __restrict__ counts, const int32_t* __restrict__ idx, int units,
+                 int NB, int causal, unsigned long long* __restrict__ order) {
   extern __shared__ int hist[];  // NB + 1 bins, bin = NB - count
   const int nbins = NB + 1;
   for (int i = threadIdx.x; i < nbins; i += kThreads) hist[i] = 0;
   __syncthreads();
-  for (int u = threadIdx.x; u < units; u += kThreads) {
-    int c = counts[u];
-    c = c < 0 ? 0 : (c > NB ? NB : c);
-    atomicAdd(&hist[NB - c], 1);
+  // 8 units per thread per batch: their load chains overlap
+  for (int u0 = 0; u0 < units; u0 += 8 * kThreads) {
+    int n[8];
+    bool diag[8];
+    unit_info8(counts, idx, u0 + threadIdx.x, units, NB, causal, n, diag);
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (u0 + threadIdx.x + q * kThreads < units) atomicAdd(&hist[NB - n[q]], 1);
   }
   __syncthreads();
   // exclusive scan of the bins: each thread sums a contiguous chunk
@@ -42,7 +91,7 @@ __global__ void __launch_bounds__(kThreads)
   if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int w = warp_tot[lane];
+    const int w = warp_tot[lane];
     int wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -59,21 +108,29 @@ __global__ void __launch_bounds__(kThreads)
     run += c;
   }
   __syncthreads();
-  for (int u = threadIdx.x; u < units; u += kThreads) {
-    int c = counts[u];
-    c = c < 0 ? 0 : (c > NB ? NB : c);
-    const int pos = atomicAdd(&hist[NB - c], 1);
-    order[pos] = static_cast<uint32_t>(u);
+  for (int u0 = 0; u0 < units; u0 += 8 * kThreads) {
+    int n[8];
+    bool diag[8];
+    unit_info8(counts, idx, u0 + threadIdx.x, units, NB, causal, n, diag);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int u = u0 + threadIdx.x + q * kThreads;
+      if (u >= units) continue;
+      const int pos = atomicAdd(&hist[NB - n[q]], 1);
+      order[pos] = static_cast<unsigned long long>(static_cast<uint32_t>(u)) |
+                   (static_cast<unsigned long long>(n[q]) << 32) |
+                   (static_cast<unsigned long long>(diag[q] ? 1 : 0) << 48);
+    }
   }
 }
 
 }  // namespace
 
-cudaError_t launch_sched(const Dims& D, const int32_t* counts, uint32_t* order,
-                         cudaStream_t st) {
+cudaError_t launch_sched(const Dims& D, const int32_t* counts, const int32_t* idx,
+                         unsigned long long* order, cudaStream_t st) {
   const int units = D.batch * D.hq * D.NB;
   const size_t smem = static_cast<size_t>(D.NB + 1) * sizeof(int);
-  sched_kernel<<<1, kThreads, smem, st>>>(counts, units, D.NB, order);
+  sched_kernel<<<1, kThreads, smem, st>>>(counts, idx, units, D.NB, D.causal, order);
   return cudaGetLastError();
 }
 

@@ -113,7 +113,7 @@ int xattn_select(const float* probs, const float* tau, const xattn_shape* shape,
 
 /*
  * Bytes of workspace xattn_sparse_attn needs (the work schedule:
- * 4 * (batch*hq*NB + 64) bytes). Returns 0 for an invalid shape.
+ * 8 * (batch*hq*NB + 32) bytes). Returns 0 for an invalid shape.
  */
 size_t xattn_attn_workspace_bytes(const xattn_shape* shape);
 
@@ -150,7 +150,7 @@ int xattn_sparse_attn(const void* Q, const void* K, const void* V, const xattn_s
  * pressure).
  *
  * The work order lives in a __device__ array of the library, sized for
- * XATTN_NOALLOC_MAX_UNITS work units (1 MiB). Each GPU that loads the library
+ * XATTN_NOALLOC_MAX_UNITS work units (2 MiB). Each GPU that loads the library
  * holds it until the process exits. Returns XATTN_ERR_WORKSPACE when
  * batch*hq*(L/B) exceeds that limit.
  *

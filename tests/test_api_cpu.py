@@ -37,7 +37,7 @@ def test_workspace_sizes(lib):
     s = X.make_shape(1, 32, 8, 131072, 128, 128, 16, True, "bf16")
     NB, r = 1024, 8
     assert X.xattn_score_workspace_bytes(s) == 32 * r * NB * (NB + 1) // 2 * 4 + 256
-    assert X.xattn_attn_workspace_bytes(s) == 4 * (32 * NB + 64)
+    assert X.xattn_attn_workspace_bytes(s) == 8 * (32 * NB + 32)
     nc = X.make_shape(1, 24, 24, 76800, 128, 128, 4, False, "bf16")
     assert X.xattn_score_workspace_bytes(nc) == 24 * (76800 // 4) * 600 * 4 + 256
     bad = X.make_shape(1, 32, 8, 1000, 128, 128, 16, True, "bf16")
