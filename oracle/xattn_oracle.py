@@ -51,6 +51,9 @@ __all__ = [
     "find_blocks", "select_blocks", "sparse_attention_head",
     "sparse_attention", "dense_attention_naive", "dense_scores",
     "antidiagonal_sums_bruteforce", "kv_head",
+    "antidiagonal_perm", "diagonal_perm", "check_perm", "top_k_blocks",
+    "top_ratio_count", "select_blocks_topk", "select_blocks_topratio",
+    "pattern_sums_bruteforce",
 ]
 
 
@@ -74,15 +77,46 @@ def kv_head(h: int, hq: int, hkv: int) -> int:
 # Step 1: strided antidiagonal reshape (§2.1; Algorithm 1, reshape loops)
 # --------------------------------------------------------------------------
 
-def reshape_queries(q: np.ndarray, S: int) -> np.ndarray:
+def antidiagonal_perm(S: int) -> list:
+    """Query sub-row of each feature chunk for the antidiagonal pattern.
+
+    Chunk i pairs query sub-row S-1-i with key sub-row i: the cells (a, b) of
+    an S x S tile with a + b = S - 1 (§2.1, lower-left to upper-right).
+    """
+    return [S - 1 - i for i in range(S)]
+
+
+def diagonal_perm(S: int) -> list:
+    """Chunk i pairs query sub-row i with key sub-row i: the main diagonal of
+    every S x S tile (the "diagonal" pattern of the sparsity-pattern ablation,
+    Knowl 9 of the chapterpal page, §3.4 Ablation Study)."""
+    return list(range(S))
+
+
+def check_perm(perm: Sequence[int], S: int) -> list:
+    """perm as a list, after checking that it is a permutation of 0..S-1."""
+    perm = [int(x) for x in perm]
+    if sorted(perm) != list(range(S)):
+        raise ValueError(f"not a permutation of 0..{S - 1}: {perm}")
+    return perm
+
+
+def reshape_queries(q: np.ndarray, S: int, perm: Sequence[int] | None = None) -> np.ndarray:
     """Q_reshaped for a slab of queries whose length is a multiple of S.
 
     The slices q[i::S] are joined along the features for i = S-1 down to 0,
     so reshaped row t is [q[tS+S-1], q[tS+S-2], ..., q[tS]].
+
+    ``perm`` generalises the order: feature chunk i holds the slice
+    q[perm[i]::S]. The default is the antidiagonal order perm[i] = S-1-i;
+    perm[i] = i gives the main diagonal, and any other permutation one cell
+    per row and per column of every S x S tile (a "random" pattern when the
+    permutation is drawn at random).
     """
     n, d = q.shape
     assert n % S == 0
-    parts = [q[i::S, :] for i in range(S - 1, -1, -1)]
+    perm = antidiagonal_perm(S) if perm is None else check_perm(perm, S)
+    parts = [q[perm[i]::S, :] for i in range(S)]
     return np.concatenate(parts, axis=1)
 
 
@@ -97,9 +131,11 @@ def reshape_keys(k: np.ndarray, S: int) -> np.ndarray:
     return np.concatenate(parts, axis=1)
 
 
-def reshaped_logits(q: np.ndarray, k: np.ndarray, S: int) -> np.ndarray:
-    """Q_r K_r^T without the 1/sqrt(d_h S) scale (the raw antidiagonal sums)."""
-    return reshape_queries(q, S) @ reshape_keys(k, S).T
+def reshaped_logits(q: np.ndarray, k: np.ndarray, S: int,
+                    perm: Sequence[int] | None = None) -> np.ndarray:
+    """Q_r K_r^T without the 1/sqrt(d_h S) scale (the raw antidiagonal sums,
+    or the sums of the pattern ``perm`` selects)."""
+    return reshape_queries(q, S, perm) @ reshape_keys(k, S).T
 
 
 # --------------------------------------------------------------------------
@@ -128,7 +164,8 @@ def approx_attention_rows(x_scaled: np.ndarray, row0: int, causal: bool) -> np.n
 
 def block_probs_head(q: np.ndarray, k: np.ndarray, B: int, S: int, causal: bool,
                      q_blocks: Iterable[int] | None = None,
-                     chunk_rows: int = 1024) -> np.ndarray:
+                     chunk_rows: int = 1024,
+                     perm: Sequence[int] | None = None) -> np.ndarray:
     """P[b, j] for one head: the normalised block sums of A_approx.
 
     q, k: [L, d] float64. Returns an [NB, NB] array. With ``q_blocks`` given,
@@ -140,12 +177,15 @@ def block_probs_head(q: np.ndarray, k: np.ndarray, B: int, S: int, causal: bool,
     multiple of S). So several blocks' reshaped logits can come from one
     matmul call. Every row is then masked, normalised and block-summed on its
     own, exactly as the per-block loop does.
+
+    ``perm`` selects the sampling pattern inside each S x S tile (see
+    reshape_queries); the default is the antidiagonal.
     """
     L, d = q.shape
     assert L % B == 0 and B % S == 0
     NB, r = L // B, B // S
     scale = 1.0 / math.sqrt(d * S)
-    Qr = reshape_queries(q, S)
+    Qr = reshape_queries(q, S, perm)
     Kr = reshape_keys(k, S)
     P = np.full((NB, NB), np.nan)
     blocks = list(range(NB)) if q_blocks is None else sorted(set(int(b) for b in q_blocks))
@@ -167,7 +207,8 @@ def block_probs_head(q: np.ndarray, k: np.ndarray, B: int, S: int, causal: bool,
 
 
 def block_probs(Q, K, B: int, S: int, causal: bool, heads: Sequence[int] | None = None,
-                q_blocks: Iterable[int] | None = None) -> np.ndarray:
+                q_blocks: Iterable[int] | None = None,
+                perm: Sequence[int] | None = None) -> np.ndarray:
     """P for [batch, hq, L, d] queries and [batch, hkv, L, d] keys.
 
     Returns [batch, hq, NB, NB]. Heads outside ``heads`` are NaN.
@@ -181,7 +222,7 @@ def block_probs(Q, K, B: int, S: int, causal: bool, heads: Sequence[int] | None 
     for bb in range(b_):
         for h in hs:
             out[bb, h] = block_probs_head(Qf[bb, h], Kf[bb, kv_head(h, hq, hkv)], B, S,
-                                          causal, q_blocks)
+                                          causal, q_blocks, perm=perm)
     return out
 
 
@@ -234,6 +275,83 @@ def select_blocks(P: np.ndarray, tau: Sequence[float], causal: bool,
                 mask[bb, h, b, sel] = True
                 lists[(bb, h, b)] = sel
     return mask, lists
+
+
+# --------------------------------------------------------------------------
+# Step 4b: fixed-budget selection, the Top-K and Top-Ratio strategies of the
+# selection-strategy ablation (Knowl 9 of the chapterpal page; §3.4 Ablation
+# Study). The pages name them only; the readings used here:
+# * both rank a row's allowed blocks like find_blocks (probability
+#   descending, ties to the lower index) and keep a fixed number of them;
+# * Top-K keeps k blocks per row (k counted in blocks; a token budget such as
+#   K = 8192 is K / B blocks), or every allowed block when fewer are allowed;
+# * Top-Ratio keeps ratio * n blocks of a row with n allowed blocks, rounded
+#   to the nearest integer (halves up), and at least one block.
+# --------------------------------------------------------------------------
+
+def top_k_blocks(p: np.ndarray, k: int) -> np.ndarray:
+    """The k allowed blocks of highest probability (ties: lower index first).
+
+    Returns ascending indices; every allowed block when k >= len(p).
+    """
+    p = np.asarray(p, dtype=np.float64)
+    n = p.shape[0]
+    if k < 1:
+        raise ValueError("k must be at least 1")
+    order = np.lexsort((np.arange(n), -p))     # primary: -p, secondary: index
+    return np.sort(order[:min(k, n)])
+
+
+def top_ratio_count(ratio: float, n: int) -> int:
+    """Blocks kept by Top-Ratio in a row with n allowed blocks.
+
+    ratio is taken as an fp32 value (the type the boundary passes). The
+    product ratio * n is exact in float64 (a 24-bit significand times an
+    integer below 2^13), and so is adding 1/2 for every ratio the count can
+    depend on, so floor(ratio * n + 1/2) is the exactly rounded count.
+    """
+    r = float(np.float32(ratio))
+    if not (0.0 < r <= 1.0):
+        raise ValueError("ratio must lie in (0, 1]")
+    k = int(math.floor(r * n + 0.5))
+    return max(1, min(n, k))
+
+
+def _select_rows(P: np.ndarray, causal: bool, heads, q_blocks, choose):
+    P = np.asarray(P, dtype=np.float64)
+    b_, hq, NB, _ = P.shape
+    mask = np.zeros(P.shape, dtype=bool)
+    lists = {}
+    hs = range(hq) if heads is None else heads
+    bs = range(NB) if q_blocks is None else q_blocks
+    for bb in range(b_):
+        for h in hs:
+            for b in bs:
+                n = b + 1 if causal else NB
+                sel = choose(P[bb, h, b, :n], h)
+                mask[bb, h, b, sel] = True
+                lists[(bb, h, b)] = sel
+    return mask, lists
+
+
+def select_blocks_topk(P: np.ndarray, k: Sequence[int], causal: bool,
+                       heads: Sequence[int] | None = None,
+                       q_blocks: Iterable[int] | None = None):
+    """Top-K on every row of P ([batch, hq, NB, NB]); k is per query head.
+
+    Returns (mask, lists) like select_blocks.
+    """
+    return _select_rows(P, causal, heads, q_blocks,
+                        lambda row, h: top_k_blocks(row, int(k[h])))
+
+
+def select_blocks_topratio(P: np.ndarray, ratio: Sequence[float], causal: bool,
+                           heads: Sequence[int] | None = None,
+                           q_blocks: Iterable[int] | None = None):
+    """Top-Ratio on every row of P; ratio is per query head, in (0, 1]."""
+    return _select_rows(
+        P, causal, heads, q_blocks,
+        lambda row, h: top_k_blocks(row, top_ratio_count(float(ratio[h]), row.shape[0])))
 
 
 # --------------------------------------------------------------------------
@@ -353,6 +471,23 @@ def antidiagonal_sums_bruteforce(q: np.ndarray, k: np.ndarray, S: int) -> np.nda
             for a in range(S):
                 for b in range(S):
                     if a + b == S - 1:
+                        acc += float(np.dot(q[t * S + a], k[c * S + b]))
+            out[t, c] = acc
+    return out
+
+
+def pattern_sums_bruteforce(q: np.ndarray, k: np.ndarray, S: int,
+                            perm: Sequence[int]) -> np.ndarray:
+    """Sum of q_a . k_b over the cells of every S x S tile that a pattern
+    samples: local offsets (a, b) with a == perm[b] (b = key offset)."""
+    n, m = q.shape[0], k.shape[0]
+    out = np.zeros((n // S, m // S))
+    for t in range(n // S):
+        for c in range(m // S):
+            acc = 0.0
+            for a in range(S):
+                for b in range(S):
+                    if a == perm[b]:
                         acc += float(np.dot(q[t * S + a], k[c * S + b]))
             out[t, c] = acc
     return out

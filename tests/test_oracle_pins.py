@@ -285,3 +285,155 @@ def test_q_block_subset_equals_full():
     part = O.block_probs_head(q, k, 64, 8, True, q_blocks=[0, 3, 7])
     for b in (0, 3, 7):
         np.testing.assert_allclose(part[b], full[b], rtol=0, atol=1e-14)
+
+
+# ------------------------------------------------- sampling patterns --------
+def _random_perm(S, seed):
+    return [int(x) for x in np.random.default_rng(seed).permutation(S)]
+
+
+@pytest.mark.parametrize("S", [1, 2, 4, 8])
+@pytest.mark.parametrize("kind", ["antidiagonal", "diagonal", "random"])
+def test_pattern_reshape_equals_bruteforce(S, kind):
+    """The generalised reshape samples exactly the cells a == perm[b] of every
+    S x S tile (query offset a, key offset b), checked cell by cell."""
+    perm = {"antidiagonal": O.antidiagonal_perm(S), "diagonal": O.diagonal_perm(S),
+            "random": _random_perm(S, S)}[kind]
+    q, k = _rand(32, 4), _rand(32, 4)
+    got = O.reshaped_logits(q, k, S, perm)
+    want = O.pattern_sums_bruteforce(q, k, S, perm)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_default_pattern_is_the_antidiagonal():
+    """No permutation means the antidiagonal (lower-left to upper-right)."""
+    q, k = _rand(32, 4), _rand(32, 4)
+    np.testing.assert_array_equal(O.reshaped_logits(q, k, 4),
+                                  O.reshaped_logits(q, k, 4, [3, 2, 1, 0]))
+    np.testing.assert_allclose(O.reshaped_logits(q, k, 4),
+                               O.antidiagonal_sums_bruteforce(q, k, 4), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("delta,seen", [(0, True), (4, True), (1, False), (3, False)])
+def test_diagonal_pattern_parity(delta, seen):
+    """The main-diagonal pattern only pairs q, k with q - k = 0 (mod S): a
+    planted slash at an offset that is a multiple of S is seen, any other is
+    not (the opposite of the antidiagonal's odd-offset rule for S = 4)."""
+    S, L, d = 4, 64, 16
+    q = np.zeros((L, d))
+    k = np.zeros((L, d))
+    for i in range(L):
+        q[i, i % d] = 1.0
+    for j in range(L):
+        if j + delta < L:
+            k[j, (j + delta) % d] = 1.0
+    x = O.reshaped_logits(q, k, S, O.diagonal_perm(S))
+    assert (np.abs(x).sum() > 0) == seen
+
+
+def test_perm_must_be_a_permutation():
+    with pytest.raises(ValueError):
+        O.reshape_queries(_rand(8, 2), 4, [0, 0, 1, 2])
+    with pytest.raises(ValueError):
+        O.reshape_queries(_rand(8, 2), 4, [0, 1, 2])
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_pattern_rows_are_distributions(causal):
+    """Any sampling pattern still gives rows of P that sum to 1, and causal P
+    is 0 above the diagonal."""
+    q, k = _rand(256, 8), _rand(256, 8)
+    P = O.block_probs_head(q, k, 32, 8, causal, perm=_random_perm(8, 7))
+    np.testing.assert_allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    if causal:
+        assert np.all(np.triu(P, 1) == 0)
+
+
+# --------------------------------------------- Top-K and Top-Ratio ----------
+def _dyadic_row(n, r):
+    """Probabilities that are multiples of 1/64 (sums are exact), with ties."""
+    return r.integers(0, 6, size=n) / 64.0
+
+
+@pytest.mark.parametrize("trial", range(30))
+def test_top_k_bruteforce(trial):
+    """Top-K keeps the k-subset with the largest sum; among those, the one
+    whose ascending index tuple is smallest (ties go to the lower index).
+    Checked against every k-subset of a small row."""
+    r = np.random.default_rng(100 + trial)
+    n = int(r.integers(1, 10))
+    p = _dyadic_row(n, r)
+    k = int(r.integers(1, n + 2))
+    got = tuple(int(x) for x in O.top_k_blocks(p, k))
+    if k >= n:
+        assert got == tuple(range(n))
+        return
+    best = None
+    for sub in itertools.combinations(range(n), k):
+        key = (-sum(p[list(sub)]), sub)
+        if best is None or key < best:
+            best = key
+    assert got == best[1]
+
+
+def test_top_k_is_the_threshold_set_of_the_same_size():
+    """For any tau, find_blocks keeps exactly the Top-K set with k = its size
+    (both rank by probability, then index)."""
+    r = np.random.default_rng(5)
+    for _ in range(50):
+        p = r.dirichlet(np.ones(40) * 0.3)
+        p[r.integers(0, 40, 5)] = p[3]  # ties
+        tau = float(r.uniform(0.1, 0.99))
+        sel = O.find_blocks(p, tau)
+        np.testing.assert_array_equal(O.top_k_blocks(p, len(sel)), sel)
+
+
+def test_top_k_rejects_nonpositive_k():
+    with pytest.raises(ValueError):
+        O.top_k_blocks(np.ones(4) / 4, 0)
+
+
+def test_top_ratio_count_exact():
+    """The rounded count equals round-half-up of the exact rational product
+    of the fp32 ratio and n (Fraction arithmetic), clamped to [1, n]."""
+    from fractions import Fraction
+    ratios = [0.27, 0.5, 0.1, 0.3, 1.0, 0.999, 1e-9, 0.0625, 0.7, 1 / 3, 0.25, 0.125]
+    for ratio in ratios:
+        fr = Fraction(float(np.float32(ratio)))
+        for n in list(range(1, 70)) + [127, 128, 255, 1000, 1024, 2048, 4095, 4096]:
+            x = fr * n
+            want = int((x + Fraction(1, 2)).__floor__())
+            want = max(1, min(n, want))
+            assert O.top_ratio_count(ratio, n) == want, (ratio, n)
+    # halves go up: 0.5 * 3 = 1.5 -> 2; 0.25 * 2 = 0.5 -> 1
+    assert O.top_ratio_count(0.5, 3) == 2
+    assert O.top_ratio_count(0.25, 2) == 1
+    assert O.top_ratio_count(0.27, 100) == 27
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_select_topk_and_topratio_rows(causal):
+    """Row counts follow min(k, allowed) and the rounded ratio; the kept
+    blocks are allowed ones and outrank every dropped allowed block."""
+    r = np.random.default_rng(11)
+    NB = 20
+    P = np.zeros((1, 2, NB, NB))
+    for h in range(2):
+        for b in range(NB):
+            n = b + 1 if causal else NB
+            P[0, h, b, :n] = r.dirichlet(np.ones(n))
+    for kind, arg in (("k", [3, 7]), ("ratio", [0.27, 0.6])):
+        if kind == "k":
+            mask, lists = O.select_blocks_topk(P, arg, causal)
+        else:
+            mask, lists = O.select_blocks_topratio(P, arg, causal)
+        for h in range(2):
+            for b in range(NB):
+                n = b + 1 if causal else NB
+                want_n = min(arg[h], n) if kind == "k" else O.top_ratio_count(arg[h], n)
+                sel = lists[(0, h, b)]
+                assert len(sel) == want_n and mask[0, h, b].sum() == want_n
+                assert np.all(sel < n)
+                dropped = np.setdiff1d(np.arange(n), sel)
+                if len(dropped):
+                    assert P[0, h, b, sel].min() >= P[0, h, b, dropped].max()
