@@ -3,12 +3,16 @@
 Three steps, each one call into the C-ABI library ``libxattn.so``:
 ``xattn_score`` (strided antidiagonal block scoring), ``xattn_select``
 (find_blocks threshold selection) and ``xattn_sparse_attn`` (block-sparse
-attention over the selected blocks). The library loads on first use and the
-calls raise if it is missing.
+attention over the selected blocks). The pages' ablation variants run
+through the same kernels: ``xattn_score_pattern`` (diagonal or random
+sampling) and ``xattn_select_topk`` / ``xattn_select_topratio`` (fixed
+budgets). The library loads on first use and the calls raise if it is
+missing.
 """
 from .xattn import (  # noqa: F401
     XattnError, xattn_score, xattn_select, xattn_sparse_attn, xattn_score_workspace_bytes,
     xattn_attn_workspace_bytes, xattn_get_device_status, xattn_strerror, make_shape,
-    library_path, EXPORTED_SYMBOLS, xattn_sparse_attn_noalloc,
+    library_path, EXPORTED_SYMBOLS, xattn_sparse_attn_noalloc, xattn_score_pattern,
+    xattn_select_topk, xattn_select_topratio, antidiagonal_perm, diagonal_perm,
 )
 from .pipeline import prefill_attention  # noqa: F401

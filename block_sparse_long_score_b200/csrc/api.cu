@@ -141,8 +141,13 @@ size_t xattn_score_workspace_bytes(const xattn_shape* shape) {
          256;
 }
 
-int xattn_score(const void* Q, const void* K, const xattn_shape* shape, float* probs, void* ws,
-                size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Scoring with an explicit sampling pattern (already validated).
+int score_impl(const void* Q, const void* K, const xattn_shape* shape, const PermArg& perm,
+               float* probs, void* ws, size_t ws_bytes, void* stream) {
   Dims D;
   int rc = check_shape(shape, &D);
   if (rc != XATTN_OK) return rc;
@@ -158,15 +163,62 @@ int xattn_score(const void* Q, const void* K, const xattn_shape* shape, float* p
     CUtensorMap tq, tk;
     if ((rc = make_map_reshaped(&tq, Q, D.S, D.R, D.batch * D.hq, 128)) != XATTN_OK) return rc;
     if ((rc = make_map_reshaped(&tk, K, D.S, D.R, D.batch * D.hkv, 256)) != XATTN_OK) return rc;
-    if ((rc = cuda_status(launch_score_tc(D, tq, tk, part, ds->status, ds->num_sms, st))) !=
-        XATTN_OK)
+    if ((rc = cuda_status(launch_score_tc(D, tq, tk, perm, part, ds->status, ds->num_sms,
+                                          st))) != XATTN_OK)
       return rc;
   } else {
     if ((rc = cuda_status(launch_score_simt(D, static_cast<const float*>(Q),
-                                            static_cast<const float*>(K), part, st))) != XATTN_OK)
+                                            static_cast<const float*>(K), perm, part, st))) !=
+        XATTN_OK)
       return rc;
   }
   return cuda_status(launch_score_reduce(D, part, probs, st));
+}
+
+// Fixed-budget selection (arguments already validated into `budget`).
+int select_budget_impl(const float* probs, const BudgetArg& budget, const Dims& D,
+                       uint32_t* mask, int32_t* counts, int32_t* idx, void* stream) {
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != XATTN_OK) return rc;
+  return cuda_status(launch_select_budget(D, probs, budget, mask, counts, idx,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+int xattn_score(const void* Q, const void* K, const xattn_shape* shape, float* probs, void* ws,
+                size_t ws_bytes, void* stream) {
+  Dims D;
+  const int rc = check_shape(shape, &D);
+  if (rc != XATTN_OK) return rc;
+  if (D.S > 256) return XATTN_ERR_UNSUPPORTED;  // S divides B <= 256 for every valid shape
+  PermArg perm;  // the antidiagonal: chunk i reads query sub-row S-1-i
+  std::memset(&perm, 0, sizeof(perm));
+  for (int i = 0; i < D.S; ++i) perm.q[i] = static_cast<uint8_t>(D.S - 1 - i);
+  return score_impl(Q, K, shape, perm, probs, ws, ws_bytes, stream);
+}
+
+int xattn_score_pattern(const void* Q, const void* K, const xattn_shape* shape,
+                        const int32_t* perm, float* probs, void* ws, size_t ws_bytes,
+                        void* stream) {
+  Dims D;
+  int rc = check_shape(shape, &D);
+  if (rc != XATTN_OK) return rc;
+  if (!perm) return XATTN_ERR_INVALID_ARG;
+  if (D.S > 256) return XATTN_ERR_UNSUPPORTED;
+  PermArg pa;
+  std::memset(&pa, 0, sizeof(pa));
+  bool seen[256] = {};
+  for (int i = 0; i < D.S; ++i) {
+    const int32_t v = perm[i];
+    if (v < 0 || v >= D.S || seen[v]) return XATTN_ERR_INVALID_ARG;
+    seen[v] = true;
+    pa.q[i] = static_cast<uint8_t>(v);
+  }
+  return score_impl(Q, K, shape, pa, probs, ws, ws_bytes, stream);
 }
 
 int xattn_select(const float* probs, const float* tau, const xattn_shape* shape, uint32_t* mask,
@@ -186,6 +238,39 @@ int xattn_select(const float* probs, const float* tau, const xattn_shape* shape,
   if ((rc = device_state(&ds)) != XATTN_OK) return rc;
   return cuda_status(
       launch_select(D, probs, ta, mask, counts, idx, static_cast<cudaStream_t>(stream)));
+}
+
+int xattn_select_topk(const float* probs, const int32_t* k, const xattn_shape* shape,
+                      uint32_t* mask, int32_t* counts, int32_t* idx, void* stream) {
+  Dims D;
+  int rc = check_shape(shape, &D);
+  if (rc != XATTN_OK) return rc;
+  if (!probs || !k || !mask || !counts || !idx) return XATTN_ERR_INVALID_ARG;
+  BudgetArg ba;
+  std::memset(&ba, 0, sizeof(ba));
+  for (int h = 0; h < D.hq; ++h) {
+    if (k[h] < 1) return XATTN_ERR_INVALID_ARG;
+    ba.k[h] = k[h];
+  }
+  ba.use_ratio = 0;
+  return select_budget_impl(probs, ba, D, mask, counts, idx, stream);
+}
+
+int xattn_select_topratio(const float* probs, const float* ratio, const xattn_shape* shape,
+                          uint32_t* mask, int32_t* counts, int32_t* idx, void* stream) {
+  Dims D;
+  int rc = check_shape(shape, &D);
+  if (rc != XATTN_OK) return rc;
+  if (!probs || !ratio || !mask || !counts || !idx) return XATTN_ERR_INVALID_ARG;
+  BudgetArg ba;
+  std::memset(&ba, 0, sizeof(ba));
+  for (int h = 0; h < D.hq; ++h) {
+    const float r = ratio[h];
+    if (!(r > 0.0f && r <= 1.0f)) return XATTN_ERR_INVALID_ARG;  // also rejects NaN
+    ba.ratio[h] = r;
+  }
+  ba.use_ratio = 1;
+  return select_budget_impl(probs, ba, D, mask, counts, idx, stream);
 }
 
 size_t xattn_attn_workspace_bytes(const xattn_shape* shape) {

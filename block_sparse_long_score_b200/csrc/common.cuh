@@ -38,16 +38,32 @@ __host__ __device__ inline size_t part_row_offset(int rho, int r, int NB, bool c
   return static_cast<size_t>(r) * b * (b + 1) / 2 + t * (b + 1);
 }
 
+// Sampling pattern of the scoring step: feature chunk i of a reshaped row
+// pairs query sub-row q[i] with key sub-row i of every S x S tile. The
+// antidiagonal is q[i] = S-1-i. Entries past S are unused.
+struct PermArg {
+  uint8_t q[256];
+};
+
+// Fixed-budget selection (Top-K / Top-Ratio): per query head either a block
+// count k, or a ratio of the row's allowed blocks.
+struct BudgetArg {
+  int32_t k[XATTN_MAX_HEADS];
+  float ratio[XATTN_MAX_HEADS];
+  int use_ratio;
+};
+
 // ------------------------------------------------------------ launchers
 // Each returns cudaSuccess or the launch error. All are asynchronous.
 
 // bf16 tensor-core scoring GEMM: partials for every (bh, rho, allowed j).
 cudaError_t launch_score_tc(const Dims& D, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                            float* part, int* status, int num_sms, cudaStream_t st);
+                            const PermArg& perm, float* part, int* status, int num_sms,
+                            cudaStream_t st);
 
 // fp32 CUDA-core scoring, same partial layout.
-cudaError_t launch_score_simt(const Dims& D, const float* Q, const float* K, float* part,
-                              cudaStream_t st);
+cudaError_t launch_score_simt(const Dims& D, const float* Q, const float* K,
+                              const PermArg& perm, float* part, cudaStream_t st);
 
 // partials -> block probabilities P [bh, NB, NB].
 cudaError_t launch_score_reduce(const Dims& D, const float* part, float* probs,
@@ -60,6 +76,11 @@ struct TauArg {
 // find_blocks on every row of P.
 cudaError_t launch_select(const Dims& D, const float* probs, const TauArg& tau, uint32_t* mask,
                           int32_t* counts, int32_t* idx, cudaStream_t st);
+
+// Top-K / Top-Ratio on every row of P (same outputs as launch_select).
+cudaError_t launch_select_budget(const Dims& D, const float* probs, const BudgetArg& budget,
+                                 uint32_t* mask, int32_t* counts, int32_t* idx,
+                                 cudaStream_t st);
 
 // Longest-list-first order of the work units (bh, b) into `order`: one packed
 // 64-bit entry per unit (unit index, effective block count, diagonal flag).

@@ -4,7 +4,8 @@
 // tensor-core kernel, so the same reduce kernel produces P.
 //
 // One CTA per (reshaped query row rho, batch*head). The reshaped query row
-// [Q[rho S + S-1], ..., Q[rho S]] is staged in shared memory. Each warp takes
+// [Q[rho S + S-1], ..., Q[rho S]] (in general [Q[rho S + q[0]], ...,
+// Q[rho S + q[S-1]]] for a pattern permutation q) is staged in shared memory. Each warp takes
 // one key block at a time; its lanes take that block's reshaped columns c,
 // whose reshaped key rows K[c S .. c S + S-1] are contiguous in memory.
 #include "common.cuh"
@@ -29,7 +30,7 @@ __device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2
 
 __global__ void __launch_bounds__(kThreads)
     score_simt_kernel(const float* __restrict__ Q, const float* __restrict__ K,
-                      float* __restrict__ part, Dims D, float sl2) {
+                      float* __restrict__ part, Dims D, float sl2, PermArg perm) {
   extern __shared__ float qr[];  // S * d
   const int rho = blockIdx.x;
   const int bh = blockIdx.y;
@@ -40,7 +41,7 @@ __global__ void __launch_bounds__(kThreads)
 
   for (int e = threadIdx.x; e < SD; e += kThreads) {
     const int i = e / D.d, f = e % D.d;
-    qr[e] = Qh[static_cast<size_t>(rho * D.S + D.S - 1 - i) * D.d + f];
+    qr[e] = Qh[static_cast<size_t>(rho * D.S + perm.q[i]) * D.d + f];
   }
   __syncthreads();
 
@@ -71,8 +72,8 @@ __global__ void __launch_bounds__(kThreads)
 
 }  // namespace
 
-cudaError_t launch_score_simt(const Dims& D, const float* Q, const float* K, float* part,
-                              cudaStream_t st) {
+cudaError_t launch_score_simt(const Dims& D, const float* Q, const float* K,
+                              const PermArg& perm, float* part, cudaStream_t st) {
   const float sl2 = static_cast<float>(1.4426950408889634 / sqrt(double(D.d) * D.S));
   const size_t smem = static_cast<size_t>(D.S) * D.d * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(score_simt_kernel,
@@ -80,7 +81,7 @@ cudaError_t launch_score_simt(const Dims& D, const float* Q, const float* K, flo
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(D.R, D.batch * D.hq);
-  score_simt_kernel<<<grid, kThreads, smem, st>>>(Q, K, part, D, sl2);
+  score_simt_kernel<<<grid, kThreads, smem, st>>>(Q, K, part, D, sl2, perm);
   return cudaGetLastError();
 }
 

@@ -8,7 +8,10 @@
 // [K[c S], ..., K[c S + S-1]], so k-chunk i (d features) of the GEMM pairs query
 // token rho S + S-1-i with key token c S + i. Neither operand is copied: Q and
 // K are read through 4-D TMA views [head][rho][s][feature], and chunk i takes
-// s = S-1-i on the query side and s = i on the key side.
+// s = S-1-i on the query side and s = i on the key side. The query sub-row of
+// each chunk comes from a permutation argument, so the same kernel also runs
+// the diagonal (s = i) and random-permutation patterns of the sparsity-pattern
+// ablation (Knowl 9 of the chapterpal page, §3.4 Ablation Study).
 //
 // Tiles are 128 (rho) x 256 (c), accumulated in TMEM (fp32), two accumulators
 // (512 columns) so the epilogue of one tile overlaps the MMAs of the next.
@@ -43,6 +46,7 @@ struct Params {
   int MT, NT, tiles_per_head;
   long long total_tiles;
   float scale_log2;     // log2(e) / sqrt(d * S)
+  PermArg perm;         // query sub-row of each key sub-row (antidiagonal: S-1-i)
   float* part;
   size_t part_head;     // floats per (batch, head)
   int* status;
@@ -222,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(&sm->empty[stage], phase ^ 1, abort)) goto producer_done;
             uint8_t* sa = stage_mem + stage * kStageBytes;
             mbar_arrive_expect_tx(&sm->full[stage], kStageBytes);
-            tma_load_4d(sa, &tmQ, &sm->full[stage], f * kBK, p.S - 1 - i, m0, bh);
+            tma_load_4d(sa, &tmQ, &sm->full[stage], f * kBK, p.perm.q[i], m0, bh);
             tma_load_4d(sa + kABytes, &tmK, &sm->full[stage], f * kBK, i, n0, kvbh);
             ++issued;
             if (++stage == kStages) {
@@ -331,8 +335,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_score_tc(const Dims& D, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                            float* part, int* status, int num_sms, cudaStream_t st) {
+                            const PermArg& perm, float* part, int* status, int num_sms,
+                            cudaStream_t st) {
   Params p{};
+  p.perm = perm;
   p.R = D.R;
   p.S = D.S;
   p.r = D.r;

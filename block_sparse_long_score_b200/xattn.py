@@ -20,6 +20,8 @@ __all__ = [
     "xattn_score_workspace_bytes", "xattn_attn_workspace_bytes",
     "xattn_get_device_status", "xattn_strerror", "make_shape", "library_path",
     "EXPORTED_SYMBOLS", "xattn_sparse_attn_noalloc", "NOALLOC_MAX_UNITS",
+    "xattn_score_pattern", "xattn_select_topk", "xattn_select_topratio",
+    "antidiagonal_perm", "diagonal_perm",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,7 +31,8 @@ XATTN_F32, XATTN_BF16 = 0, 1
 EXPORTED_SYMBOLS = (
     "xattn_score_workspace_bytes", "xattn_score", "xattn_select",
     "xattn_attn_workspace_bytes", "xattn_sparse_attn", "xattn_get_device_status",
-    "xattn_strerror", "xattn_sparse_attn_noalloc",
+    "xattn_strerror", "xattn_sparse_attn_noalloc", "xattn_score_pattern",
+    "xattn_select_topk", "xattn_select_topratio",
 )
 # batch * hq * (L / B) limit of xattn_sparse_attn_noalloc (XATTN_NOALLOC_MAX_UNITS)
 NOALLOC_MAX_UNITS = 1 << 18
@@ -71,6 +74,15 @@ def _lib() -> ctypes.CDLL:
         lib.xattn_score.restype = i32
         lib.xattn_select.argtypes = [vp, ctypes.POINTER(ctypes.c_float), sp, vp, vp, vp, vp]
         lib.xattn_select.restype = i32
+        lib.xattn_score_pattern.argtypes = [vp, vp, sp, ctypes.POINTER(ctypes.c_int32), vp, vp,
+                                            sz, vp]
+        lib.xattn_score_pattern.restype = i32
+        lib.xattn_select_topk.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), sp, vp, vp, vp,
+                                          vp]
+        lib.xattn_select_topk.restype = i32
+        lib.xattn_select_topratio.argtypes = [vp, ctypes.POINTER(ctypes.c_float), sp, vp, vp,
+                                              vp, vp]
+        lib.xattn_select_topratio.restype = i32
         lib.xattn_sparse_attn.argtypes = [vp, vp, vp, sp, vp, vp, vp, vp, vp, sz, vp]
         lib.xattn_sparse_attn.restype = i32
         lib.xattn_sparse_attn_noalloc.argtypes = [vp, vp, vp, sp, vp, vp, vp, vp, vp]
@@ -129,10 +141,24 @@ def xattn_attn_workspace_bytes(shape: _Shape) -> int:
     return int(_lib().xattn_attn_workspace_bytes(ctypes.byref(shape)))
 
 
+def antidiagonal_perm(S: int) -> list:
+    """Sampling pattern of xattn_score: chunk i reads query sub-row S-1-i."""
+    return [S - 1 - i for i in range(S)]
+
+
+def diagonal_perm(S: int) -> list:
+    """Main-diagonal sampling pattern: chunk i reads query sub-row i."""
+    return list(range(S))
+
+
 def xattn_score(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal: bool,
                 probs: Optional[torch.Tensor] = None,
-                workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Block probabilities P [batch, hq, L/B, L/B] (fp32) of antidiagonal scoring."""
+                workspace: Optional[torch.Tensor] = None,
+                perm: Optional[Sequence[int]] = None) -> torch.Tensor:
+    """Block probabilities P [batch, hq, L/B, L/B] (fp32) of antidiagonal scoring.
+
+    With ``perm`` (a permutation of 0..S-1) the call is xattn_score_pattern:
+    chunk i pairs query sub-row perm[i] with key sub-row i."""
     _check(Q, "Q")
     _check(K, "K", Q.dtype)
     shape = _shape_of(Q, K, B, S, causal)
@@ -144,24 +170,36 @@ def xattn_score(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal: bool,
     if workspace is None:
         workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
     _check(workspace, "workspace")
-    rc = _lib().xattn_score(Q.data_ptr(), K.data_ptr(), ctypes.byref(shape), probs.data_ptr(),
-                            workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                            _stream(Q.device))
-    _raise("xattn_score", rc)
+    if perm is None:
+        rc = _lib().xattn_score(Q.data_ptr(), K.data_ptr(), ctypes.byref(shape),
+                                probs.data_ptr(), workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size(), _stream(Q.device))
+        _raise("xattn_score", rc)
+    else:
+        perm = [int(x) for x in perm]
+        if len(perm) != S:
+            raise ValueError("perm needs S entries")
+        parr = (ctypes.c_int32 * S)(*perm)
+        rc = _lib().xattn_score_pattern(Q.data_ptr(), K.data_ptr(), ctypes.byref(shape), parr,
+                                        probs.data_ptr(), workspace.data_ptr(),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(Q.device))
+        _raise("xattn_score_pattern", rc)
     return probs
 
 
-def xattn_select(probs: torch.Tensor, tau: Sequence[float], causal: bool,
-                 out: Optional[tuple] = None):
-    """find_blocks on every row of P. Returns (mask uint32 [.., NB, ceil(NB/32)] as
-    int32, counts int32 [.., NB], idx int32 [.., NB, NB])."""
+def xattn_score_pattern(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal: bool,
+                        perm: Sequence[int], probs: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Scoring with the sampling pattern ``perm`` (see xattn_score)."""
+    return xattn_score(Q, K, B, S, causal, probs=probs, workspace=workspace, perm=perm)
+
+
+def _select_outputs(probs: torch.Tensor, causal: bool, out: Optional[tuple]):
     _check(probs, "probs", torch.float32)
     b, hq, NB, NB2 = probs.shape
     if NB != NB2:
         raise ValueError("probs must be [batch, hq, NB, NB]")
-    taus = [float(t) for t in tau]
-    if len(taus) != hq:
-        raise ValueError("tau needs one value per query head")
     shape = make_shape(b, hq, hq, NB, 128, 1, 1, causal, XATTN_F32)
     W = (NB + 31) // 32
     if out is None:
@@ -172,10 +210,51 @@ def xattn_select(probs: torch.Tensor, tau: Sequence[float], causal: bool,
         mask, counts, idx = out
     for t, n in ((mask, "mask"), (counts, "counts"), (idx, "idx")):
         _check(t, n, torch.int32)
-    tarr = (ctypes.c_float * hq)(*taus)
+    return shape, mask, counts, idx
+
+
+def _per_head(values, hq: int, name: str, kind):
+    vals = [kind(v) for v in values]
+    if len(vals) != hq:
+        raise ValueError(f"{name} needs one value per query head")
+    return vals
+
+
+def xattn_select(probs: torch.Tensor, tau: Sequence[float], causal: bool,
+                 out: Optional[tuple] = None):
+    """find_blocks on every row of P. Returns (mask uint32 [.., NB, ceil(NB/32)] as
+    int32, counts int32 [.., NB], idx int32 [.., NB, NB])."""
+    shape, mask, counts, idx = _select_outputs(probs, causal, out)
+    taus = _per_head(tau, shape.hq, "tau", float)
+    tarr = (ctypes.c_float * shape.hq)(*taus)
     rc = _lib().xattn_select(probs.data_ptr(), tarr, ctypes.byref(shape), mask.data_ptr(),
                              counts.data_ptr(), idx.data_ptr(), _stream(probs.device))
     _raise("xattn_select", rc)
+    return mask, counts, idx
+
+
+def xattn_select_topk(probs: torch.Tensor, k: Sequence[int], causal: bool,
+                      out: Optional[tuple] = None):
+    """Top-K: the k[h] best allowed blocks of every row (outputs as xattn_select)."""
+    shape, mask, counts, idx = _select_outputs(probs, causal, out)
+    ks = _per_head(k, shape.hq, "k", int)
+    karr = (ctypes.c_int32 * shape.hq)(*ks)
+    rc = _lib().xattn_select_topk(probs.data_ptr(), karr, ctypes.byref(shape), mask.data_ptr(),
+                                  counts.data_ptr(), idx.data_ptr(), _stream(probs.device))
+    _raise("xattn_select_topk", rc)
+    return mask, counts, idx
+
+
+def xattn_select_topratio(probs: torch.Tensor, ratio: Sequence[float], causal: bool,
+                          out: Optional[tuple] = None):
+    """Top-Ratio: round(ratio[h] * allowed) best blocks of every row (at least one)."""
+    shape, mask, counts, idx = _select_outputs(probs, causal, out)
+    rs = _per_head(ratio, shape.hq, "ratio", float)
+    rarr = (ctypes.c_float * shape.hq)(*rs)
+    rc = _lib().xattn_select_topratio(probs.data_ptr(), rarr, ctypes.byref(shape),
+                                      mask.data_ptr(), counts.data_ptr(), idx.data_ptr(),
+                                      _stream(probs.device))
+    _raise("xattn_select_topratio", rc)
     return mask, counts, idx
 
 

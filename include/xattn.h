@@ -28,6 +28,11 @@
  *   that exceeded its time limit) are recorded in a per-device status word
  *   that xattn_get_device_status reads and clears. Kernels never trap.
  *
+ * Two further calls run the pages' ablation variants through the same
+ * kernels: xattn_score_pattern (diagonal / random sampling instead of the
+ * antidiagonal) and xattn_select_topk / xattn_select_topratio (fixed budgets
+ * instead of the threshold).
+ *
  * Data types: XATTN_BF16 runs the tensor-core (tcgen05) kernels and needs
  * d = 128 and B = 128. XATTN_F32 runs plain FP32 CUDA-core kernels for small
  * problems and needs d in {32, 64, 128} and B <= 256.
@@ -110,6 +115,46 @@ int xattn_score(const void* Q, const void* K, const xattn_shape* shape, float* p
  */
 int xattn_select(const float* probs, const float* tau, const xattn_shape* shape,
                  uint32_t* mask, int32_t* counts, int32_t* idx, void* stream);
+
+/*
+ * Scoring with another sampling pattern inside each S x S tile: the
+ * sparsity-pattern ablation of "XAttention: Block Sparse Attention with
+ * Antidiagonal Scoring" (chapterpal page, Knowl 9; §3.4 Ablation Study)
+ * compares the antidiagonal with diagonal and random sampling.
+ *
+ * perm: HOST pointer to S int32 values, a permutation of 0..S-1. Feature
+ *       chunk i of a reshaped row pairs query token rho*S + perm[i] with key
+ *       token c*S + i, so the score of tile (rho, c) is the sum of q.k over
+ *       the cells (perm[i], i). perm[i] = S-1-i is the antidiagonal (equal to
+ *       xattn_score), perm[i] = i the main diagonal; a random pattern is a
+ *       permutation the caller draws. INVALID_ARG if perm is NULL or not a
+ *       permutation.
+ * Everything else (scale, causal mask, softmax, block sums, probs, workspace,
+ * errors) is as for xattn_score.
+ */
+int xattn_score_pattern(const void* Q, const void* K, const xattn_shape* shape,
+                        const int32_t* perm, float* probs, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/*
+ * Fixed-budget selection, the Top-K and Top-Ratio strategies of the
+ * selection-strategy ablation (chapterpal page, Knowl 9; §3.4 Ablation Study).
+ * A row's allowed blocks (0..b when causal, all NB otherwise; n of them) are
+ * ranked as in xattn_select (probability descending, index ascending) and the
+ * first k are kept:
+ *   xattn_select_topk:     k = min(k[h], n). k: HOST pointer to hq int32
+ *                          values, each >= 1 (a token budget K is K / B blocks).
+ *   xattn_select_topratio: k = ratio[h] * n rounded to the nearest integer
+ *                          (halves up), at least 1 and at most n. ratio: HOST
+ *                          pointer to hq floats in (0, 1]. The product is
+ *                          formed exactly, so the count is exact.
+ * Outputs (mask, counts, idx) have the layout of xattn_select. INVALID_ARG for
+ * a NULL pointer or a k / ratio out of range.
+ */
+int xattn_select_topk(const float* probs, const int32_t* k, const xattn_shape* shape,
+                      uint32_t* mask, int32_t* counts, int32_t* idx, void* stream);
+int xattn_select_topratio(const float* probs, const float* ratio, const xattn_shape* shape,
+                          uint32_t* mask, int32_t* counts, int32_t* idx, void* stream);
 
 /*
  * Bytes of workspace xattn_sparse_attn needs (the work schedule:

@@ -91,3 +91,44 @@ def test_strerror(lib):
     assert X.xattn_strerror(0) == "ok"
     assert "timed out" in X.xattn_strerror(-5)
     assert X.xattn_strerror(42) == "unknown status"
+
+
+@pytest.mark.parametrize("perm", [[0, 0, 1, 2, 3, 4, 5, 6], [0, 1, 2, 3, 4, 5, 6, 8],
+                                  [-1, 1, 2, 3, 4, 5, 6, 7], None])
+def test_bad_pattern_rejected(lib, perm):
+    s = X.make_shape(1, 4, 2, 1024, 128, 128, 8, True, "bf16")
+    arr = None if perm is None else (ctypes.c_int32 * 8)(*perm)
+    assert lib.xattn_score_pattern(FAKE, FAKE, ctypes.byref(s), arr, FAKE, FAKE, 1 << 40,
+                                   None) == -1
+
+
+def test_pattern_checks_shape_and_workspace_first(lib):
+    ok = (ctypes.c_int32 * 8)(*range(8))
+    bad = X.make_shape(1, 4, 2, 1000, 128, 128, 8, True, "bf16")
+    assert lib.xattn_score_pattern(FAKE, FAKE, ctypes.byref(bad), ok, FAKE, FAKE, 1 << 40,
+                                   None) == -1
+    s = X.make_shape(1, 4, 2, 1024, 128, 128, 8, True, "bf16")
+    assert lib.xattn_score_pattern(FAKE, FAKE, ctypes.byref(s), ok, FAKE, FAKE, 16, None) == -4
+
+
+@pytest.mark.parametrize("k", [0, -3])
+def test_topk_out_of_range(lib, k):
+    s = X.make_shape(1, 2, 2, 1024, 128, 128, 8, True, "bf16")
+    arr = (ctypes.c_int32 * 2)(4, k)
+    assert lib.xattn_select_topk(FAKE, arr, ctypes.byref(s), FAKE, FAKE, FAKE, None) == -1
+
+
+@pytest.mark.parametrize("ratio", [0.0, -0.1, 1.5, float("nan")])
+def test_topratio_out_of_range(lib, ratio):
+    s = X.make_shape(1, 2, 2, 1024, 128, 128, 8, True, "bf16")
+    arr = (ctypes.c_float * 2)(0.25, ratio)
+    assert lib.xattn_select_topratio(FAKE, arr, ctypes.byref(s), FAKE, FAKE, FAKE, None) == -1
+
+
+def test_budget_null_pointers(lib):
+    s = X.make_shape(1, 2, 2, 1024, 128, 128, 8, True, "bf16")
+    k = (ctypes.c_int32 * 2)(4, 4)
+    r = (ctypes.c_float * 2)(0.5, 0.5)
+    assert lib.xattn_select_topk(None, k, ctypes.byref(s), FAKE, FAKE, FAKE, None) == -1
+    assert lib.xattn_select_topk(FAKE, None, ctypes.byref(s), FAKE, FAKE, FAKE, None) == -1
+    assert lib.xattn_select_topratio(FAKE, r, ctypes.byref(s), FAKE, None, FAKE, None) == -1
