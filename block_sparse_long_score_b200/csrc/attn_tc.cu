@@ -198,36 +198,45 @@ __device__ __forceinline__ bool event_s(SlotState& st, Ring& ring, const Ctx& x)
   const bool last = c.j == c.n - 1;
   if (!kMma) {
     if (first) {
-      if (!mbar_wait(&sm->q_empty[kSlot], (st.units & 1) ^ 1, x.abort)) return false;
-      mbar_arrive_expect_tx(&sm->q_full[kSlot], kTileBytes);
-      const int qrow = c.bh * p.L + c.qb * kBlk;
-      tma_load_2d(x.q_smem + kSlot * kTileBytes, x.tmQ, &sm->q_full[kSlot], 0, qrow);
-      tma_load_2d(x.q_smem + kSlot * kTileBytes + kHalf, x.tmQ, &sm->q_full[kSlot], 64, qrow);
+      if (!warp_wait(&sm->q_empty[kSlot], (st.units & 1) ^ 1, x.abort)) return false;
+      if (elect_one()) {
+        mbar_arrive_expect_tx(&sm->q_full[kSlot], kTileBytes);
+        const int qrow = c.bh * p.L + c.qb * kBlk;
+        tma_load_2d(x.q_smem + kSlot * kTileBytes, x.tmQ, &sm->q_full[kSlot], 0, qrow);
+        tma_load_2d(x.q_smem + kSlot * kTileBytes + kHalf, x.tmQ, &sm->q_full[kSlot], 64, qrow);
+      }
+      __syncwarp();
     }
-    if (!mbar_wait(&sm->kv_empty[ring.stage], ring.phase ^ 1, x.abort)) return false;
-    const int kvbh = (c.bh / p.hq) * p.hkv + (c.bh % p.hq) / p.group;
-    const int krow = kvbh * p.L + c.kb * kBlk;
-    uint8_t* dst = x.kv_smem + ring.stage * kTileBytes;
-    mbar_arrive_expect_tx(&sm->kv_full[ring.stage], kTileBytes);
-    tma_load_2d(dst, x.tmK, &sm->kv_full[ring.stage], 0, krow);
-    tma_load_2d(dst + kHalf, x.tmK, &sm->kv_full[ring.stage], 64, krow);
+    if (!warp_wait(&sm->kv_empty[ring.stage], ring.phase ^ 1, x.abort)) return false;
+    if (elect_one()) {
+      const int kvbh = (c.bh / p.hq) * p.hkv + (c.bh % p.hq) / p.group;
+      const int krow = kvbh * p.L + c.kb * kBlk;
+      uint8_t* dst = x.kv_smem + ring.stage * kTileBytes;
+      mbar_arrive_expect_tx(&sm->kv_full[ring.stage], kTileBytes);
+      tma_load_2d(dst, x.tmK, &sm->kv_full[ring.stage], 0, krow);
+      tma_load_2d(dst + kHalf, x.tmK, &sm->kv_full[ring.stage], 64, krow);
+    }
+    __syncwarp();
     ++ring.issued;
   } else {
-    if (first && !mbar_wait(&sm->q_full[kSlot], st.units & 1, x.abort)) return false;
-    if (!mbar_wait(&sm->kv_full[ring.stage], ring.phase, x.abort)) return false;
+    if (first && !warp_wait(&sm->q_full[kSlot], st.units & 1, x.abort)) return false;
+    if (!warp_wait(&sm->kv_full[ring.stage], ring.phase, x.abort)) return false;
     tc_fence_after();
-    const uint32_t q_addr = smem_u32(x.q_smem + kSlot * kTileBytes);
-    const uint32_t k_addr = smem_u32(x.kv_smem + ring.stage * kTileBytes);
-    const uint32_t dS = x.tmem + kSlot * kSlotCols;
+    if (elect_one()) {
+      const uint32_t q_addr = smem_u32(x.q_smem + kSlot * kTileBytes);
+      const uint32_t k_addr = smem_u32(x.kv_smem + ring.stage * kTileBytes);
+      const uint32_t dS = x.tmem + kSlot * kSlotCols;
 #pragma unroll
-    for (int kk = 0; kk < kD / 16; ++kk) {
-      const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-      umma_ss(dS, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
-              kIdescS, kk > 0);
+      for (int kk = 0; kk < kD / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+        umma_ss(dS, smem_desc_sw128(q_addr + off, 16, 1024),
+                smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0);
+      }
+      umma_commit(&sm->s_full[kSlot]);
+      umma_commit(&sm->kv_empty[ring.stage]);
+      if (last) umma_commit(&sm->q_empty[kSlot]);
     }
-    umma_commit(&sm->s_full[kSlot]);
-    umma_commit(&sm->kv_empty[ring.stage]);
-    if (last) umma_commit(&sm->q_empty[kSlot]);
+    __syncwarp();
   }
   if (first) ++st.units;
   st.pend = true;
@@ -245,31 +254,37 @@ __device__ __forceinline__ bool event_pv(SlotState& st, Ring& ring, const Ctx& x
   const Cursor& c = st.cur;
   const bool first = st.pend_j == 0;
   if (!kMma) {
-    if (!mbar_wait(&sm->kv_empty[ring.stage], ring.phase ^ 1, x.abort)) return false;
-    const int kvbh = (c.bh / p.hq) * p.hkv + (c.bh % p.hq) / p.group;
-    const int vrow = kvbh * p.L + c.kb * kBlk;
-    uint8_t* dst = x.kv_smem + ring.stage * kTileBytes;
-    mbar_arrive_expect_tx(&sm->kv_full[ring.stage], kTileBytes);
-    tma_load_2d(dst, x.tmV, &sm->kv_full[ring.stage], 0, vrow);
-    tma_load_2d(dst + kHalf, x.tmV, &sm->kv_full[ring.stage], 64, vrow);
+    if (!warp_wait(&sm->kv_empty[ring.stage], ring.phase ^ 1, x.abort)) return false;
+    if (elect_one()) {
+      const int kvbh = (c.bh / p.hq) * p.hkv + (c.bh % p.hq) / p.group;
+      const int vrow = kvbh * p.L + c.kb * kBlk;
+      uint8_t* dst = x.kv_smem + ring.stage * kTileBytes;
+      mbar_arrive_expect_tx(&sm->kv_full[ring.stage], kTileBytes);
+      tma_load_2d(dst, x.tmV, &sm->kv_full[ring.stage], 0, vrow);
+      tma_load_2d(dst + kHalf, x.tmV, &sm->kv_full[ring.stage], 64, vrow);
+    }
+    __syncwarp();
     ++ring.issued;
   } else {
-    if (!mbar_wait(&sm->p_full[kSlot], st.blocks & 1, x.abort)) return false;
+    if (!warp_wait(&sm->p_full[kSlot], st.blocks & 1, x.abort)) return false;
     // the unit's first PV overwrites O: the previous unit's epilogue must be done
-    if (first && !mbar_wait(&sm->o_empty[kSlot], ((st.units - 1) & 1) ^ 1, x.abort)) return false;
-    if (!mbar_wait(&sm->kv_full[ring.stage], ring.phase, x.abort)) return false;
+    if (first && !warp_wait(&sm->o_empty[kSlot], ((st.units - 1) & 1) ^ 1, x.abort)) return false;
+    if (!warp_wait(&sm->kv_full[ring.stage], ring.phase, x.abort)) return false;
     tc_fence_after();
-    const uint32_t v_addr = smem_u32(x.kv_smem + ring.stage * kTileBytes);
-    const uint32_t dO = x.tmem + kSlot * kSlotCols + kColO;
-    const uint32_t aP = x.tmem + kSlot * kSlotCols;
+    if (elect_one()) {
+      const uint32_t v_addr = smem_u32(x.kv_smem + ring.stage * kTileBytes);
+      const uint32_t dO = x.tmem + kSlot * kSlotCols + kColO;
+      const uint32_t aP = x.tmem + kSlot * kSlotCols;
 #pragma unroll
-    for (int kk = 0; kk < kBlk / 16; ++kk) {
-      // 16 keys per step: P columns [8kk, 8kk+8) (bf16 pairs), V rows [16kk, 16kk+16)
-      umma_ts(dO, aP + kk * 8, smem_desc_sw128(v_addr + kk * 16 * 128, kHalf, 1024), kIdescPV,
-              (!first || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < kBlk / 16; ++kk) {
+        // 16 keys per step: P columns [8kk, 8kk+8) (bf16 pairs), V rows [16kk, 16kk+16)
+        umma_ts(dO, aP + kk * 8, smem_desc_sw128(v_addr + kk * 16 * 128, kHalf, 1024), kIdescPV,
+                (!first || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(&sm->pv_done[kSlot]);
+      umma_commit(&sm->kv_empty[ring.stage]);
     }
-    umma_commit(&sm->pv_done[kSlot]);
-    umma_commit(&sm->kv_empty[ring.stage]);
+    __syncwarp();
   }
   ++st.blocks;
   st.pend = false;
@@ -369,9 +384,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");  // 128 x 80
-    if (warp <= 1 && lane == 0) {
+    if (warp <= 1) {
       // Producer (warp 0) and MMA issuer (warp 1) walk the same merged event
       // order: S(0), S(1), { PV(0), S(0, next), PV(1), S(1, next) } ...
+      // Each role runs on its whole warp; one elected lane issues the TMA
+      // copies / MMAs and commits.
       if (warp == 0)
         pipeline<false>(p, sm, q_smem, kv_smem, tmem, &tmQ, &tmK, &tmV, abort);
       else

@@ -71,6 +71,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// One lane of a converged warp (the lowest active one) gets true. Issuing
+// roles run their bookkeeping on the whole warp, which keeps it in uniform
+// registers, and let the elected lane issue the single-thread tcgen05 / TMA
+// instructions; a loop run by one lane alone issues tensor-core work much
+// more slowly.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .b32 %%rx;\n\t.reg .pred %%px;\n\t"
+      "elect.sync %%rx|%%px, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, %%px;\n\t}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // All 32 lanes wait; the result is the same on every lane (false if any lane
 // gave up), so warp-collective tcgen05 instructions after it stay converged.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {

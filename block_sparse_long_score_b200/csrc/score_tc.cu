@@ -21,8 +21,8 @@
 // are skipped.
 //
 // Warp roles (256 threads, 1 CTA per SM, persistent over tiles):
-//   warp 0      TMA producer (one thread)
-//   warp 1      TMEM allocator + MMA issuer (one thread)
+//   warp 0      TMA producer (one elected lane issues the copies)
+//   warp 1      TMEM allocator + MMA issuer (one elected lane issues the MMAs)
 //   warps 4..7  epilogue, one TMEM lane (= one reshaped row) per thread
 #include "common.cuh"
 #include "ptx.cuh"
@@ -210,8 +210,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm->tmem_base;
   volatile int* abort = &sm->abort;
 
+  // The producer and MMA roles run on whole warps (bookkeeping stays warp-
+  // uniform); one elected lane issues each TMA copy, MMA and commit.
   if (warp == 0) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------ TMA producer
       int stage = 0;
       uint32_t phase = 0;
@@ -223,11 +225,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int m0 = mt * kBM, n0 = nt * kBN;
         for (int i = 0; i < p.S; ++i) {
           for (int f = 0; f < 2; ++f) {
-            if (!mbar_wait(&sm->empty[stage], phase ^ 1, abort)) goto producer_done;
-            uint8_t* sa = stage_mem + stage * kStageBytes;
-            mbar_arrive_expect_tx(&sm->full[stage], kStageBytes);
-            tma_load_4d(sa, &tmQ, &sm->full[stage], f * kBK, p.perm.q[i], m0, bh);
-            tma_load_4d(sa + kABytes, &tmK, &sm->full[stage], f * kBK, i, n0, kvbh);
+            if (!warp_wait(&sm->empty[stage], phase ^ 1, abort)) goto producer_done;
+            if (elect_one()) {
+              uint8_t* sa = stage_mem + stage * kStageBytes;
+              mbar_arrive_expect_tx(&sm->full[stage], kStageBytes);
+              tma_load_4d(sa, &tmQ, &sm->full[stage], f * kBK, p.perm.q[i], m0, bh);
+              tma_load_4d(sa + kABytes, &tmK, &sm->full[stage], f * kBK, i, n0, kvbh);
+            }
+            __syncwarp();
             ++issued;
             if (++stage == kStages) {
               stage = 0;
@@ -252,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------ MMA issuer
       int stage = 0;
       uint32_t phase = 0;
@@ -260,33 +265,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (long long t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++it) {
         const int buf = it & 1;
         const uint32_t aph = (it >> 1) & 1;
-        if (!mbar_wait(&sm->acc_empty[buf], aph ^ 1, abort)) break;
+        if (!warp_wait(&sm->acc_empty[buf], aph ^ 1, abort)) break;
         tc_fence_after();
         const uint32_t dacc = tmem + buf * kBN;
         const int ksteps = 2 * p.S;
         bool ok = true;
         for (int ks = 0; ks < ksteps; ++ks) {
-          if (!mbar_wait(&sm->full[stage], phase, abort)) {
+          if (!warp_wait(&sm->full[stage], phase, abort)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(stage_mem + stage * kStageBytes);
-          const uint32_t sb = sa + kABytes;
+          if (elect_one()) {
+            const uint32_t sa = smem_u32(stage_mem + stage * kStageBytes);
+            const uint32_t sb = sa + kABytes;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t da = smem_desc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t db = smem_desc_sw128(sb + kk * 32, 16, 1024);
-            umma_ss(dacc, da, db, kIdesc, (ks | kk) != 0);
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t da = smem_desc_sw128(sa + kk * 32, 16, 1024);
+              const uint64_t db = smem_desc_sw128(sb + kk * 32, 16, 1024);
+              umma_ss(dacc, da, db, kIdesc, (ks | kk) != 0);
+            }
+            umma_commit(&sm->empty[stage]);
           }
-          umma_commit(&sm->empty[stage]);
+          __syncwarp();
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        umma_commit(&sm->acc_full[buf]);
+        if (elect_one()) umma_commit(&sm->acc_full[buf]);
+        __syncwarp();
       }
     }
   } else if (warp >= 4) {
