@@ -34,6 +34,19 @@ METRIC = "prefill attn ms/layer at 128K (score+select+sparse); dense-equiv TFLOP
 WORKLOAD = "c2"   # the 128K Llama-shaped layer the metric is quoted on
 
 
+# DRAM traffic (ncu dram__bytes_read.sum + dram__bytes_write.sum) per call of
+# the current kernels, for the workloads where a capture exists. The captures
+# ran the 8-query-head case of the same layer (bench.py --heads 8: 2 of the 8
+# KV groups, every query block); traffic grows with the number of heads, so the
+# figures are scaled by 32 / 8 to a full call. Summaries: profiles/.
+TRAFFIC_BYTES = {
+    # score_tc 357.72 MB read + 120.54 MB written; score_reduce 134.38 + 18.69 MB
+    ("c2", "score"): 4 * (357.72 + 120.54 + 134.38 + 18.69) * 1e6,
+    # attn_tc 850.92 MB read + 235.76 MB written (sched_kernel: 1.12 MB)
+    ("c2", "sparse_attn"): 4 * (850.92 + 235.76 + 1.12) * 1e6,
+}
+
+
 def peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -288,6 +301,14 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     dense = dense_equiv_flops(prob)
     dense_tflops = dense / (ms_step * 1e-3) / 1e12
     peak_attn = pk["bf16_sustained"]
+    # the roofline object describes the call with the largest share of the step
+    if per["score"] >= per["sparse_attn"]:
+        dom, dom_tflops = "score", score_tflops
+        dom_kernel = "xattn_score (score_tc_kernel + score_reduce_kernel)"
+    else:
+        dom, dom_tflops = "sparse_attn", attn_tflops
+        dom_kernel = "xattn_sparse_attn (sched_kernel + attn_tc_kernel)"
+    traffic = None if args.heads else TRAFFIC_BYTES.get((args.config, dom))
     line = {
         "metric": METRIC,
         "value": whole_job_ms_per_layer(ms_step, world),
@@ -314,12 +335,12 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
         },
         "roofline": {
             "bound": "tensor",
-            "kernel": "attn_tc_kernel (xattn_sparse_attn; includes the LPT schedule kernel)",
-            "achieved": attn_tflops,
+            "kernel": dom_kernel,
+            "achieved": dom_tflops,
             "peak": peak_attn,
             "unit": "TFLOP/s",
-            "frac": attn_tflops / peak_attn,
-            "traffic": None,
+            "frac": dom_tflops / peak_attn,
+            "traffic": traffic,
             "peak_source": f"{pk['source']} bf16 sustained (kernel timed inside a long step)",
         },
         "e2e": {
