@@ -145,20 +145,25 @@ size_t xattn_score_workspace_bytes(const xattn_shape* shape) {
 
 namespace {
 
-// Scoring with an explicit sampling pattern (already validated).
-int score_impl(const void* Q, const void* K, const xattn_shape* shape, const PermArg& perm,
-               float* probs, void* ws, size_t ws_bytes, void* stream) {
-  Dims D;
-  int rc = check_shape(shape, &D);
+// Host checks shared by the scoring calls (Q, K, workspace). probs may be
+// required or optional.
+int check_score_args(const void* Q, const void* K, const xattn_shape* shape, void* ws,
+                     size_t ws_bytes, Dims* D) {
+  int rc = check_shape(shape, D);
   if (rc != XATTN_OK) return rc;
-  if (!Q || !K || !probs) return XATTN_ERR_INVALID_ARG;
+  if (!Q || !K) return XATTN_ERR_INVALID_ARG;
   const size_t need = xattn_score_workspace_bytes(shape);
   if (!ws || ws_bytes < need) return XATTN_ERR_WORKSPACE;
-  if (D.dtype == XATTN_BF16 && (!aligned16(Q) || !aligned16(K))) return XATTN_ERR_INVALID_ARG;
+  if (D->dtype == XATTN_BF16 && (!aligned16(Q) || !aligned16(K))) return XATTN_ERR_INVALID_ARG;
+  return XATTN_OK;
+}
+
+// Launches the scoring GEMM (partial log-sum-exp into the workspace).
+int score_partials(const void* Q, const void* K, const Dims& D, const PermArg& perm,
+                   float* part, cudaStream_t st) {
   DeviceState* ds = nullptr;
-  if ((rc = device_state(&ds)) != XATTN_OK) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* part = static_cast<float*>(ws);
+  int rc = device_state(&ds);
+  if (rc != XATTN_OK) return rc;
   if (D.dtype == XATTN_BF16) {
     CUtensorMap tq, tk;
     if ((rc = make_map_reshaped(&tq, Q, D.S, D.R, D.batch * D.hq, 128)) != XATTN_OK) return rc;
@@ -172,7 +177,31 @@ int score_impl(const void* Q, const void* K, const xattn_shape* shape, const Per
         XATTN_OK)
       return rc;
   }
+  return XATTN_OK;
+}
+
+// Scoring with an explicit sampling pattern (already validated).
+int score_impl(const void* Q, const void* K, const xattn_shape* shape, const PermArg& perm,
+               float* probs, void* ws, size_t ws_bytes, void* stream) {
+  Dims D;
+  int rc = check_score_args(Q, K, shape, ws, ws_bytes, &D);
+  if (rc != XATTN_OK) return rc;
+  if (!probs) return XATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* part = static_cast<float*>(ws);
+  if ((rc = score_partials(Q, K, D, perm, part, st)) != XATTN_OK) return rc;
   return cuda_status(launch_score_reduce(D, part, probs, st));
+}
+
+// Per-head thresholds from a host array; INVALID_ARG unless each is in (0, 1].
+int tau_arg(const float* tau, int hq, TauArg* ta) {
+  std::memset(ta, 0, sizeof(*ta));
+  for (int h = 0; h < hq; ++h) {
+    const float t = tau[h];
+    if (!(t > 0.0f && t <= 1.0f)) return XATTN_ERR_INVALID_ARG;  // also rejects NaN
+    ta->v[h] = t;
+  }
+  return XATTN_OK;
 }
 
 // Fixed-budget selection (arguments already validated into `budget`).
@@ -228,16 +257,30 @@ int xattn_select(const float* probs, const float* tau, const xattn_shape* shape,
   if (rc != XATTN_OK) return rc;
   if (!probs || !tau || !mask || !counts || !idx) return XATTN_ERR_INVALID_ARG;
   TauArg ta;
-  std::memset(&ta, 0, sizeof(ta));
-  for (int h = 0; h < D.hq; ++h) {
-    const float t = tau[h];
-    if (!(t > 0.0f && t <= 1.0f)) return XATTN_ERR_INVALID_ARG;  // also rejects NaN
-    ta.v[h] = t;
-  }
+  if ((rc = tau_arg(tau, D.hq, &ta)) != XATTN_OK) return rc;
   DeviceState* ds = nullptr;
   if ((rc = device_state(&ds)) != XATTN_OK) return rc;
   return cuda_status(
       launch_select(D, probs, ta, mask, counts, idx, static_cast<cudaStream_t>(stream)));
+}
+
+int xattn_score_select(const void* Q, const void* K, const xattn_shape* shape, const float* tau,
+                       float* probs, uint32_t* mask, int32_t* counts, int32_t* idx, void* ws,
+                       size_t ws_bytes, void* stream) {
+  Dims D;
+  int rc = check_score_args(Q, K, shape, ws, ws_bytes, &D);
+  if (rc != XATTN_OK) return rc;
+  if (!tau || !mask || !counts || !idx) return XATTN_ERR_INVALID_ARG;
+  TauArg ta;
+  if ((rc = tau_arg(tau, D.hq, &ta)) != XATTN_OK) return rc;
+  if (D.S > 256) return XATTN_ERR_UNSUPPORTED;  // S divides B <= 256 for every valid shape
+  PermArg perm;  // the antidiagonal
+  std::memset(&perm, 0, sizeof(perm));
+  for (int i = 0; i < D.S; ++i) perm.q[i] = static_cast<uint8_t>(D.S - 1 - i);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* part = static_cast<float*>(ws);
+  if ((rc = score_partials(Q, K, D, perm, part, st)) != XATTN_OK) return rc;
+  return cuda_status(launch_score_select(D, part, probs, ta, mask, counts, idx, st));
 }
 
 int xattn_select_topk(const float* probs, const int32_t* k, const xattn_shape* shape,

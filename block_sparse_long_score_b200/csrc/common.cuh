@@ -77,6 +77,12 @@ struct TauArg {
 cudaError_t launch_select(const Dims& D, const float* probs, const TauArg& tau, uint32_t* mask,
                           int32_t* counts, int32_t* idx, cudaStream_t st);
 
+// partials -> P (optional) and find_blocks, fused (same outputs as
+// launch_score_reduce followed by launch_select).
+cudaError_t launch_score_select(const Dims& D, const float* part, float* probs,
+                                const TauArg& tau, uint32_t* mask, int32_t* counts, int32_t* idx,
+                                cudaStream_t st);
+
 // Top-K / Top-Ratio on every row of P (same outputs as launch_select).
 cudaError_t launch_select_budget(const Dims& D, const float* probs, const BudgetArg& budget,
                                  uint32_t* mask, int32_t* counts, int32_t* idx,

@@ -21,7 +21,7 @@ __all__ = [
     "xattn_get_device_status", "xattn_strerror", "make_shape", "library_path",
     "EXPORTED_SYMBOLS", "xattn_sparse_attn_noalloc", "NOALLOC_MAX_UNITS",
     "xattn_score_pattern", "xattn_select_topk", "xattn_select_topratio",
-    "antidiagonal_perm", "diagonal_perm",
+    "antidiagonal_perm", "diagonal_perm", "xattn_score_select",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -32,7 +32,7 @@ EXPORTED_SYMBOLS = (
     "xattn_score_workspace_bytes", "xattn_score", "xattn_select",
     "xattn_attn_workspace_bytes", "xattn_sparse_attn", "xattn_get_device_status",
     "xattn_strerror", "xattn_sparse_attn_noalloc", "xattn_score_pattern",
-    "xattn_select_topk", "xattn_select_topratio",
+    "xattn_select_topk", "xattn_select_topratio", "xattn_score_select",
 )
 # batch * hq * (L / B) limit of xattn_sparse_attn_noalloc (XATTN_NOALLOC_MAX_UNITS)
 NOALLOC_MAX_UNITS = 1 << 18
@@ -77,6 +77,9 @@ def _lib() -> ctypes.CDLL:
         lib.xattn_score_pattern.argtypes = [vp, vp, sp, ctypes.POINTER(ctypes.c_int32), vp, vp,
                                             sz, vp]
         lib.xattn_score_pattern.restype = i32
+        lib.xattn_score_select.argtypes = [vp, vp, sp, ctypes.POINTER(ctypes.c_float), vp, vp,
+                                           vp, vp, vp, sz, vp]
+        lib.xattn_score_select.restype = i32
         lib.xattn_select_topk.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), sp, vp, vp, vp,
                                           vp]
         lib.xattn_select_topk.restype = i32
@@ -231,6 +234,44 @@ def xattn_select(probs: torch.Tensor, tau: Sequence[float], causal: bool,
                              counts.data_ptr(), idx.data_ptr(), _stream(probs.device))
     _raise("xattn_select", rc)
     return mask, counts, idx
+
+
+def xattn_score_select(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal: bool,
+                       tau: Sequence[float], probs: Optional[torch.Tensor] | bool = None,
+                       out: Optional[tuple] = None, workspace: Optional[torch.Tensor] = None):
+    """Scoring and find_blocks in one call (P stays on chip). Returns (mask,
+    counts, idx), or (probs, mask, counts, idx) when probs is True or a tensor."""
+    _check(Q, "Q")
+    _check(K, "K", Q.dtype)
+    shape = _shape_of(Q, K, B, S, causal)
+    NB = shape.L // max(shape.B, 1)
+    want_p = probs is not None and probs is not False
+    if probs is True:
+        probs = torch.empty(shape.batch, shape.hq, NB, NB, device=Q.device, dtype=torch.float32)
+    if want_p:
+        _check(probs, "probs", torch.float32)
+    W = (NB + 31) // 32
+    if out is None:
+        mask = torch.empty(shape.batch, shape.hq, NB, W, device=Q.device, dtype=torch.int32)
+        counts = torch.empty(shape.batch, shape.hq, NB, device=Q.device, dtype=torch.int32)
+        idx = torch.empty(shape.batch, shape.hq, NB, NB, device=Q.device, dtype=torch.int32)
+    else:
+        mask, counts, idx = out
+    for t, n in ((mask, "mask"), (counts, "counts"), (idx, "idx")):
+        _check(t, n, torch.int32)
+    taus = _per_head(tau, shape.hq, "tau", float)
+    tarr = (ctypes.c_float * shape.hq)(*taus)
+    need = xattn_score_workspace_bytes(shape)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
+    _check(workspace, "workspace")
+    rc = _lib().xattn_score_select(Q.data_ptr(), K.data_ptr(), ctypes.byref(shape), tarr,
+                                   probs.data_ptr() if want_p else None, mask.data_ptr(),
+                                   counts.data_ptr(), idx.data_ptr(), workspace.data_ptr(),
+                                   workspace.numel() * workspace.element_size(),
+                                   _stream(Q.device))
+    _raise("xattn_score_select", rc)
+    return (probs, mask, counts, idx) if want_p else (mask, counts, idx)
 
 
 def xattn_select_topk(probs: torch.Tensor, k: Sequence[int], causal: bool,

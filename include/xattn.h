@@ -117,6 +117,24 @@ int xattn_select(const float* probs, const float* tau, const xattn_shape* shape,
                  uint32_t* mask, int32_t* counts, int32_t* idx, void* stream);
 
 /*
+ * xattn_score and xattn_select in one call: the scoring GEMM, then one kernel
+ * that reduces each query block's partials to its row of P and runs
+ * find_blocks on it straight from on-chip memory, so P makes no round trip
+ * through HBM (§2.2: block scores, then the threshold selection).
+ *
+ * tau:   HOST pointer to hq floats in (0, 1], as for xattn_select.
+ * probs: out, optional (may be NULL): fp32 [batch, hq, NB, NB], bit-identical
+ *        to xattn_score's output when given.
+ * mask, counts, idx: out, as for xattn_select, and bit-identical to
+ *        xattn_select run on xattn_score's P.
+ * ws / ws_bytes: the scoring workspace (xattn_score_workspace_bytes).
+ * Errors: as for xattn_score and xattn_select.
+ */
+int xattn_score_select(const void* Q, const void* K, const xattn_shape* shape, const float* tau,
+                       float* probs, uint32_t* mask, int32_t* counts, int32_t* idx, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/*
  * Scoring with another sampling pattern inside each S x S tile: the
  * sparsity-pattern ablation of "XAttention: Block Sparse Attention with
  * Antidiagonal Scoring" (chapterpal page, Knowl 9; §3.4 Ablation Study)

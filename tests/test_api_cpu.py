@@ -132,3 +132,17 @@ def test_budget_null_pointers(lib):
     assert lib.xattn_select_topk(None, k, ctypes.byref(s), FAKE, FAKE, FAKE, None) == -1
     assert lib.xattn_select_topk(FAKE, None, ctypes.byref(s), FAKE, FAKE, FAKE, None) == -1
     assert lib.xattn_select_topratio(FAKE, r, ctypes.byref(s), FAKE, None, FAKE, None) == -1
+
+
+def test_score_select_host_checks(lib):
+    s = X.make_shape(1, 2, 2, 1024, 128, 128, 8, True, "bf16")
+    good = (ctypes.c_float * 2)(0.9, 0.9)
+    bad = (ctypes.c_float * 2)(0.9, 1.5)
+    f = lib.xattn_score_select
+    assert f(FAKE, FAKE, ctypes.byref(s), bad, None, FAKE, FAKE, FAKE, FAKE, 1 << 40, None) == -1
+    assert f(FAKE, FAKE, ctypes.byref(s), None, None, FAKE, FAKE, FAKE, FAKE, 1 << 40, None) == -1
+    assert f(FAKE, FAKE, ctypes.byref(s), good, None, None, FAKE, FAKE, FAKE, 1 << 40, None) == -1
+    assert f(None, FAKE, ctypes.byref(s), good, None, FAKE, FAKE, FAKE, FAKE, 1 << 40, None) == -1
+    assert f(FAKE, FAKE, ctypes.byref(s), good, None, FAKE, FAKE, FAKE, FAKE, 16, None) == -4
+    odd = ctypes.c_void_p(0x10008)
+    assert f(odd, FAKE, ctypes.byref(s), good, None, FAKE, FAKE, FAKE, FAKE, 1 << 40, None) == -1
