@@ -196,7 +196,7 @@ def problem_overrides(args) -> dict:
 # ----------------------------------------------------------------- main arm
 def run_ours(args, rank: int, world: int, local: int) -> None:
     from block_sparse_long_score_b200 import (xattn_score, xattn_select, xattn_sparse_attn,
-                                              xattn_get_device_status,
+                                              xattn_score_select, xattn_get_device_status,
                                               xattn_score_workspace_bytes,
                                               xattn_attn_workspace_bytes, make_shape)
     from block_sparse_long_score_b200.synth import make_problem
@@ -224,10 +224,18 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        xattn_score(Q, K, prob.B, prob.S, prob.causal, probs=probs, workspace=ws_s)
-        if ev:
-            ev[1].record(stream)
-        xattn_select(probs, taus, prob.causal, out=(mask, counts, idx))
+        if args.fused:
+            # scoring, block sums and find_blocks in one call (P stays on chip);
+            # its time is reported under "score", "select" is 0
+            xattn_score_select(Q, K, prob.B, prob.S, prob.causal, taus,
+                               out=(mask, counts, idx), workspace=ws_s)
+            if ev:
+                ev[1].record(stream)
+        else:
+            xattn_score(Q, K, prob.B, prob.S, prob.causal, probs=probs, workspace=ws_s)
+            if ev:
+                ev[1].record(stream)
+            xattn_select(probs, taus, prob.causal, out=(mask, counts, idx))
         if ev:
             ev[2].record(stream)
         xattn_sparse_attn(Q, K, V, counts, idx, prob.B, prob.causal, out=out, workspace=ws_a)
@@ -297,18 +305,19 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     score_tflops = score_flops / (per["score"] * 1e-3) / 1e12
     sel_bytes = 4.0 * pairs + 4.0 * selected + 4.0 * W * NB * prob.hq * prob.batch + \
         4.0 * NB * prob.hq * prob.batch
-    sel_gbs = sel_bytes / (per["select"] * 1e-3) / 1e9
+    sel_gbs = sel_bytes / (per["select"] * 1e-3) / 1e9 if not args.fused else None
     dense = dense_equiv_flops(prob)
     dense_tflops = dense / (ms_step * 1e-3) / 1e12
     peak_attn = pk["bf16_sustained"]
     # the roofline object describes the call with the largest share of the step
     if per["score"] >= per["sparse_attn"]:
         dom, dom_tflops = "score", score_tflops
-        dom_kernel = "xattn_score (score_tc_kernel + score_reduce_kernel)"
+        dom_kernel = ("xattn_score_select (score_tc_kernel + score_select_kernel)" if args.fused
+                      else "xattn_score (score_tc_kernel + score_reduce_kernel)")
     else:
         dom, dom_tflops = "sparse_attn", attn_tflops
         dom_kernel = "xattn_sparse_attn (sched_kernel + attn_tc_kernel)"
-    traffic = None if args.heads else TRAFFIC_BYTES.get((args.config, dom))
+    traffic = None if (args.heads or args.fused) else TRAFFIC_BYTES.get((args.config, dom))
     line = {
         "metric": METRIC,
         "value": whole_job_ms_per_layer(ms_step, world),
@@ -322,7 +331,9 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded Llama-3.1-8B-shaped Q/K/V with planted sinks and slash bands)",
-        "config": workload_config(prob),
+        "config": dict(workload_config(prob),
+                       path="xattn_score_select + xattn_sparse_attn" if args.fused
+                       else "xattn_score + xattn_select + xattn_sparse_attn"),
         "dense_equiv_tflops": dense_tflops,
         "pct_peak": 100.0 * dense_tflops / pk["bf16"],
         "density": density,
@@ -330,7 +341,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
         "score_select_share": (per["score"] + per["select"]) / ms_step,
         "kernel_fracs": {
             "score": {"tflops": score_tflops, "frac": score_tflops / pk["bf16_sustained"]},
-            "select": {"gbs": sel_gbs, "frac": sel_gbs / pk["hbm_gbs"]},
+            "select": {"gbs": sel_gbs, "frac": sel_gbs / pk["hbm_gbs"] if sel_gbs else None},
             "sparse_attn": {"tflops": attn_tflops, "frac": attn_tflops / peak_attn},
         },
         "roofline": {
@@ -349,7 +360,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
             "h2d_bytes_per_step": int(Q.numel() * 2 + K.numel() * 2 + V.numel() * 2),
             "d2h_bytes_per_step": int(out.numel() * 2),
         },
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": (4 if args.fused else 5) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -398,6 +409,8 @@ def main() -> None:
     ap.add_argument("--config", default=WORKLOAD, choices=["c1", "c2", "c3", "c4"],
                     help="workload (default c2, the 128K layer the metric is quoted on)")
     ap.add_argument("--stride", type=int, default=0, help="stride S for the video layer (c4)")
+    ap.add_argument("--fused", action="store_true",
+                    help="run scoring and selection as one call (xattn_score_select)")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling case: keep this many query heads (default: all 32)")
     args = ap.parse_args()

@@ -16,7 +16,7 @@
 namespace xattn {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 128;
 
 __global__ void __launch_bounds__(kThreads)
     score_select_kernel(const float* __restrict__ part, float* __restrict__ probs,

@@ -1,7 +1,8 @@
 """The whole prefill attention step of one layer: score, select, attend.
 
-This strings the three C-ABI calls together on the current CUDA stream. It
-holds no arithmetic of its own.
+This strings the C-ABI calls together on the current CUDA stream: scoring
+fused with the block sums and find_blocks (xattn_score_select), then the
+block-sparse attention. It holds no arithmetic of its own.
 """
 from __future__ import annotations
 
@@ -9,7 +10,7 @@ from typing import Sequence
 
 import torch
 
-from .xattn import xattn_score, xattn_select, xattn_sparse_attn
+from .xattn import xattn_score_select, xattn_sparse_attn
 
 
 def prefill_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, B: int, S: int,
@@ -20,8 +21,10 @@ def prefill_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, B: int,
     dtype). tau: one threshold per query head. Returns O, or
     (O, probs, mask, counts, idx) with return_all.
     """
-    probs = xattn_score(Q, K, B, S, causal)
-    mask, counts, idx = xattn_select(probs, tau, causal)
+    if return_all:
+        probs, mask, counts, idx = xattn_score_select(Q, K, B, S, causal, tau, probs=True)
+    else:
+        mask, counts, idx = xattn_score_select(Q, K, B, S, causal, tau)
     O = xattn_sparse_attn(Q, K, V, counts, idx, B, causal)
     if return_all:
         return O, probs, mask, counts, idx
