@@ -446,19 +446,21 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (c * 32 + i > row) sv[c][i] = __float_as_uint(-INFINITY);
         }
         {
-          // 8 independent partial maxima: a short dependency chain
+          // 8 independent partial maxima over 16 scores each (three-input
+          // max: 8 instructions a group), then a short tree
           float pm[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) pm[q] = __uint_as_float(sv[q >> 1][(q & 1) * 16]);
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t* g16 = &sv[q >> 1][(q & 1) * 16];
+            float m = fmax3(__uint_as_float(g16[0]), __uint_as_float(g16[1]),
+                            __uint_as_float(g16[2]));
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int q = c * 2 + (i >> 4);
-              if ((i & 15) != 0) pm[q] = fmaxf(pm[q], __uint_as_float(sv[c][i]));
-            }
-          mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                     fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+            for (int i = 3; i < 15; i += 2)
+              m = fmax3(m, __uint_as_float(g16[i]), __uint_as_float(g16[i + 1]));
+            pm[q] = fmaxf(m, __uint_as_float(g16[15]));
+          }
+          mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]),
+                     fmaxf(pm[6], pm[7]));
         }
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool need = m_new > m_run + kRescaleLog2;

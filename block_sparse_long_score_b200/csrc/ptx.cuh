@@ -71,6 +71,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// max(a, b, c) in one instruction (the three-input form of max.f32).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // One lane of a converged warp (the lowest active one) gets true. Issuing
 // roles run their bookkeeping on the whole warp, which keeps it in uniform
 // registers, and let the elected lane issue the single-thread tcgen05 / TMA
