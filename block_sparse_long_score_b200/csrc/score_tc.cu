@@ -20,10 +20,12 @@
 // into block probabilities. Causal tiles entirely above the reshaped diagonal
 // are skipped.
 //
-// Warp roles (256 threads, 1 CTA per SM, persistent over tiles):
+// Warp roles (384 threads, 1 CTA per SM, persistent over tiles):
 //   warp 0      TMA producer (one elected lane issues the copies)
 //   warp 1      TMEM allocator + MMA issuer (one elected lane issues the MMAs)
-//   warps 4..7  epilogue, one TMEM lane (= one reshaped row) per thread
+//   warps 4..11 epilogue, one TMEM lane (= one reshaped row) per thread;
+//               warps 4..7 reduce columns 0..127 of a tile, warps 8..11 columns
+//               128..255 (a key block never straddles the halves: r divides 128)
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -37,7 +39,8 @@ constexpr int kStages = 4;
 constexpr int kABytes = kBM * kBK * 2;   // 16 KB
 constexpr int kBBytes = kBN * kBK * 2;   // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kThreads = 256;
+constexpr int kEpiWarps = 8;       // two epilogue warpgroups, one per 128-column half
+constexpr int kThreads = 128 + kEpiWarps * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN, 0, 0);
 
@@ -115,9 +118,11 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], int c0, 
     for (int g = 0; g < 32 / RP; ++g) {
       const int j = (c0 + g * RP) / RP;
       if (j > jmax) continue;
-      float m = -INFINITY;
+      float m = x[g * RP];
+      if constexpr (RP == 2) m = fmaxf(m, x[g * RP + 1]);
 #pragma unroll
-      for (int i = 0; i < RP; ++i) m = fmaxf(m, x[g * RP + i]);
+      for (int i = 1; i + 1 < RP; i += 2) m = fmax3(m, x[g * RP + i], x[g * RP + i + 1]);
+      if constexpr (RP > 2 && (RP % 2) == 0) m = fmaxf(m, x[g * RP + RP - 1]);
       if (m == -INFINITY) {  // no visible column (cannot happen for j <= jmax)
         prow[j] = -INFINITY;
         continue;
@@ -129,9 +134,10 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], int c0, 
       prow[j] = mb + lg2(s);
     }
   } else {
-    float m = -INFINITY;
+    float m = x[0];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) m = fmaxf(m, x[i]);
+    for (int i = 1; i < 31; i += 2) m = fmax3(m, x[i], x[i + 1]);
+    m = fmaxf(m, x[31]);
     const float mb = m * sl2;
     float s = 0.f;
     if (m != -INFINITY) {
@@ -157,10 +163,11 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], int c0, 
 template <int RP>
 __device__ __forceinline__ void epilogue_tile(uint32_t tacc, int rho, int n0, const Params& p,
                                               float* prow, int jmax, bool row_ok,
-                                              bool need_mask) {
+                                              bool need_mask, int half) {
   float m_run = -INFINITY, s_run = 0.f;
+  constexpr int kHalfChunks = kBN / 64;  // 32-column chunks per half tile
 #pragma unroll 1
-  for (int ch = 0; ch < kBN / 32; ++ch) {
+  for (int ch = half * kHalfChunks; ch < (half + 1) * kHalfChunks; ++ch) {
     uint32_t v[32];
     tmem_ld32(tacc + ch * 32, v);
     tmem_ld_wait();
@@ -191,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm->acc_full[b], 1);
-      mbar_init(&sm->acc_empty[b], 128);
+      mbar_init(&sm->acc_empty[b], kEpiWarps * 32);
     }
     sm->abort = 0;
     fence_barrier_init();
@@ -300,6 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4) {
     // -------------------------------------------------------- epilogue
+    // warps 4..7 take columns 0..127 of the tile, warps 8..11 columns 128..255
+    const int half = (warp - 4) / 4;
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int it = 0;
@@ -320,14 +329,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool need_mask = (n0 + kBN > p.R) || (p.causal && n0 + kBN - 1 > m0);
       const uint32_t tacc = tmem + lane_addr + buf * kBN;
       switch (p.r) {
-        case 1: epilogue_tile<1>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask); break;
-        case 2: epilogue_tile<2>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask); break;
-        case 4: epilogue_tile<4>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask); break;
-        case 8: epilogue_tile<8>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask); break;
-        case 16: epilogue_tile<16>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask); break;
-        case 32: epilogue_tile<32>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask); break;
-        case 64: epilogue_tile<64>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask); break;
-        default: epilogue_tile<128>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask); break;
+        case 1: epilogue_tile<1>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask, half); break;
+        case 2: epilogue_tile<2>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask, half); break;
+        case 4: epilogue_tile<4>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask, half); break;
+        case 8: epilogue_tile<8>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask, half); break;
+        case 16: epilogue_tile<16>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask, half); break;
+        case 32: epilogue_tile<32>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask, half); break;
+        case 64: epilogue_tile<64>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask, half); break;
+        default: epilogue_tile<128>(tacc, rho, n0, p, prow, jmax, row_ok, need_mask, half); break;
       }
       tc_fence_before();
       mbar_arrive(&sm->acc_empty[buf]);
