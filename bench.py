@@ -40,10 +40,10 @@ WORKLOAD = "c2"   # the 128K Llama-shaped layer the metric is quoted on
 # KV groups, every query block); traffic grows with the number of heads, so the
 # figures are scaled by 32 / 8 to a full call. Summaries: profiles/.
 TRAFFIC_BYTES = {
-    # score_tc 357.72 MB read + 120.54 MB written; score_reduce 134.38 + 18.69 MB
-    ("c2", "score"): 4 * (357.72 + 120.54 + 134.38 + 18.69) * 1e6,
-    # attn_tc 850.92 MB read + 235.76 MB written (sched_kernel: 1.12 MB)
-    ("c2", "sparse_attn"): 4 * (850.92 + 235.76 + 1.12) * 1e6,
+    # score_tc 358.13 MB read + 120.59 MB written; score_reduce 134.38 + 19.69 MB
+    ("c2", "score"): 4 * (358.13 + 120.59 + 134.38 + 19.69) * 1e6,
+    # attn_tc 841.86 MB read + 237.50 MB written (sched_kernel: 1.12 MB)
+    ("c2", "sparse_attn"): 4 * (841.86 + 237.50 + 1.12) * 1e6,
 }
 
 
