@@ -198,14 +198,19 @@ def _video(cfg: dict, frames: int, frame_tokens: int, hq: int, seed: int) -> tup
 def make_problem(name: str, *, L: int | None = None, hq: int | None = None,
                  hkv: int | None = None, S: int | None = None, frames: int | None = None,
                  frame_tokens: int | None = None, seed: int | None = None,
-                 tau: float | None = None, gamma: float | None = None) -> Problem:
+                 tau: float | None = None, gamma: float | None = None,
+                 batch: int | None = None) -> Problem:
     """Build one workload by name ("c0".."c4").
 
     The keyword overrides shrink a workload for tests: same recipe, fewer
-    tokens or heads. For "c4", S picks one stride of the sweep (default 8),
+    tokens or heads (or more sequences: ``batch``). For "c4", S picks one stride of the sweep (default 8),
     and ``frames`` and ``frame_tokens`` set L.
     """
     cfg = dict(CONFIGS[name])
+    if batch is not None:
+        if cfg["kind"] == "tiny" and batch != 1:
+            raise ValueError("the tiny fp32 workload has one sequence")
+        cfg["batch"] = int(batch)
     seed = cfg["seed"] if seed is None else seed
     hq = cfg["hq"] if hq is None else hq
     hkv = cfg["hkv"] if hkv is None else hkv

@@ -218,3 +218,54 @@ def test_full_size_sampled(name, kw, heads):
     if prob.causal:
         assert np.all(res["P"][0, :, np.triu_indices(prob.NB, 1)[0], np.triu_indices(prob.NB, 1)[1]] == 0)
     check_problem(prob, heads, sample_blocks(prob.NB), res)
+
+
+# ------------------------------------------------------------- batch > 1 ----
+def test_batch_of_two_every_path():
+    """Two sequences in one call: every batch element checked against the
+    oracle (P, masks, outputs), through the three calls, the fused call and
+    the no-alloc attention."""
+    from block_sparse_long_score_b200 import xattn_score_select, xattn_sparse_attn_noalloc
+    prob = make_problem("c1", L=2048, hq=4, hkv=2, batch=2)
+    assert prob.Q.shape[0] == 2
+    Q, K, V = prob.Q.to(DEV), prob.K.to(DEV), prob.V.to(DEV)
+    taus = prob.tau.tolist()
+    P = xattn_score(Q, K, prob.B, prob.S, prob.causal)
+    mask, counts, idx = xattn_select(P, taus, prob.causal)
+    out, lse = xattn_sparse_attn(Q, K, V, counts, idx, prob.B, prob.causal, lse=True)
+    P2, mask2, counts2, idx2 = xattn_score_select(Q, K, prob.B, prob.S, prob.causal, taus,
+                                                  probs=True)
+    out2 = torch.empty_like(Q)
+    xattn_sparse_attn_noalloc(Q, K, V, counts, idx, prob.B, prob.causal, out2)
+    torch.cuda.synchronize()
+    assert xattn_get_device_status() == 0
+    assert torch.equal(P, P2) and torch.equal(mask, mask2) and torch.equal(counts, counts2)
+    assert torch.equal(out, out2)
+    Pn, mb = PT.to_np(P), PT.mask_to_bool(PT.to_np(mask), prob.NB)
+    cn, ixn = PT.to_np(counts), PT.to_np(idx)
+    On, ln = PT.to_np(out.float()), PT.to_np(lse)
+    P_ref = O.block_probs(prob.Q, prob.K, prob.B, prob.S, prob.causal)
+    lists = {}
+    for bb in range(2):
+        for h in range(prob.hq):
+            assert PT.check_probs(Pn[bb, h], P_ref[bb, h]) <= 1.0
+            for b in range(prob.NB):
+                bd, _, _ = PT.compare_row_masks(P_ref[bb, h, b], float(taus[h]), b + 1, mb[bb, h, b])
+                assert bd == 0, (bb, h, b)
+                lists[(bb, h, b)] = [int(x) for x in ixn[bb, h, b, : cn[bb, h, b]]]
+    Oref, lref = O.sparse_attention(prob.Q, prob.K, prob.V, prob.B, prob.causal, lists)
+    assert np.max(np.abs(On - Oref)) <= PT.O_TOL["bf16"]
+    assert np.max(np.abs(ln - lref)) <= PT.LSE_TOL["bf16"]
+    # the two sequences differ, so a batch-index mix-up would show
+    assert np.max(np.abs(On[0] - On[1])) > 0.1
+
+
+# -------------------------------------------------------- maximum size ----
+def test_maximum_block_count():
+    """NB = 4096 query / key blocks (L = 512K tokens, the largest NB the calls
+    accept), one head: sampled query blocks against the oracle."""
+    prob = make_problem("c1", L=4096 * 128, hq=1, hkv=1)
+    assert prob.NB == 4096
+    res = run_gpu(prob)
+    qblocks = [0, 1, 2047, 3000, 4094, 4095]
+    check_problem(prob, [0], qblocks, res)
