@@ -14,6 +14,6 @@ from .xattn import (  # noqa: F401
     xattn_attn_workspace_bytes, xattn_get_device_status, xattn_strerror, make_shape,
     library_path, EXPORTED_SYMBOLS, xattn_sparse_attn_noalloc, xattn_score_pattern,
     xattn_select_topk, xattn_select_topratio, antidiagonal_perm, diagonal_perm,
-    xattn_score_select,
+    xattn_score_select, xattn_selftest_timeout,
 )
 from .pipeline import prefill_attention  # noqa: F401

@@ -355,6 +355,13 @@ int xattn_sparse_attn(const void* Q, const void* K, const void* V, const xattn_s
                                       static_cast<float*>(O), lse, st));
 }
 
+int xattn_selftest_timeout(void* stream) {
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != XATTN_OK) return rc;
+  return cuda_status(launch_selftest_timeout(ds->status, static_cast<cudaStream_t>(stream)));
+}
+
 int xattn_get_device_status(void* stream) {
   DeviceState* ds = nullptr;
   int rc = device_state(&ds);

@@ -83,6 +83,9 @@ cudaError_t launch_score_select(const Dims& D, const float* part, float* probs,
                                 const TauArg& tau, uint32_t* mask, int32_t* counts, int32_t* idx,
                                 cudaStream_t st);
 
+// One CTA whose bounded wait runs out (failure-detection self-test).
+cudaError_t launch_selftest_timeout(int* status, cudaStream_t st);
+
 // Top-K / Top-Ratio on every row of P (same outputs as launch_select).
 cudaError_t launch_select_budget(const Dims& D, const float* probs, const BudgetArg& budget,
                                  uint32_t* mask, int32_t* counts, int32_t* idx,

@@ -21,7 +21,7 @@ __all__ = [
     "xattn_get_device_status", "xattn_strerror", "make_shape", "library_path",
     "EXPORTED_SYMBOLS", "xattn_sparse_attn_noalloc", "NOALLOC_MAX_UNITS",
     "xattn_score_pattern", "xattn_select_topk", "xattn_select_topratio",
-    "antidiagonal_perm", "diagonal_perm", "xattn_score_select",
+    "antidiagonal_perm", "diagonal_perm", "xattn_score_select", "xattn_selftest_timeout",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -33,6 +33,7 @@ EXPORTED_SYMBOLS = (
     "xattn_attn_workspace_bytes", "xattn_sparse_attn", "xattn_get_device_status",
     "xattn_strerror", "xattn_sparse_attn_noalloc", "xattn_score_pattern",
     "xattn_select_topk", "xattn_select_topratio", "xattn_score_select",
+    "xattn_selftest_timeout",
 )
 # batch * hq * (L / B) limit of xattn_sparse_attn_noalloc (XATTN_NOALLOC_MAX_UNITS)
 NOALLOC_MAX_UNITS = 1 << 18
@@ -90,6 +91,8 @@ def _lib() -> ctypes.CDLL:
         lib.xattn_sparse_attn.restype = i32
         lib.xattn_sparse_attn_noalloc.argtypes = [vp, vp, vp, sp, vp, vp, vp, vp, vp]
         lib.xattn_sparse_attn_noalloc.restype = i32
+        lib.xattn_selftest_timeout.argtypes = [vp]
+        lib.xattn_selftest_timeout.restype = i32
         lib.xattn_get_device_status.argtypes = [vp]
         lib.xattn_get_device_status.restype = i32
         lib.xattn_strerror.argtypes = [i32]
@@ -354,6 +357,12 @@ def xattn_sparse_attn_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                                           _stream(Q.device))
     _raise("xattn_sparse_attn_noalloc", rc)
     return out
+
+
+def xattn_selftest_timeout(device=None) -> None:
+    """Launches the failure-detection self-test (see include/xattn.h): the next
+    xattn_get_device_status on this stream returns XATTN_ERR_TIMEOUT."""
+    _raise("xattn_selftest_timeout", _lib().xattn_selftest_timeout(_stream(device)))
 
 
 def xattn_get_device_status(device=None) -> int:

@@ -235,6 +235,17 @@ int xattn_sparse_attn_noalloc(const void* Q, const void* K, const void* V,
  */
 int xattn_get_device_status(void* stream);
 
+/*
+ * Self-test of the failure detection: launches one small kernel whose
+ * bounded pipeline wait (the same wait every kernel of the library uses) runs
+ * out after its time limit (about 2 s), because nothing ever completes the
+ * barrier it waits on. The kernel records the time-out in the device status
+ * word and returns normally, so the next xattn_get_device_status on the stream
+ * returns XATTN_ERR_TIMEOUT and clears it, and the context stays usable. No
+ * fault, trap or unbounded wait is involved. Returns XATTN_OK once launched.
+ */
+int xattn_selftest_timeout(void* stream);
+
 /* Static, human-readable text for an xattn_status value. */
 const char* xattn_strerror(int status);
 
