@@ -67,6 +67,7 @@ struct Params {
   __nv_bfloat16* O;
   float* lse;
   int* status;
+  int o_store32;  // O is 32-byte aligned: rows are written with 32-byte stores
 };
 
 struct Smem {
@@ -536,9 +537,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           w[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv, __uint_as_float(v[2 * i + 1]) * inv);
-        uint4* dst = reinterpret_cast<uint4*>(optr + c * 32);
+        if (p.o_store32) {
+          // full 32-byte sectors, half the store instructions
+          st_global_v8(optr + c * 32, w);
+          st_global_v8(optr + c * 32 + 16, w + 8);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(optr + c * 32);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
       }
       if (p.lse) p.lse[orow] = (m_run + lg2(l_run)) * 0.69314718055994531f;
       tc_fence_before();
@@ -574,6 +582,7 @@ cudaError_t launch_attn_tc(const Dims& D, const CUtensorMap& tmQ, const CUtensor
   p.O = static_cast<__nv_bfloat16*>(O);
   p.lse = lse;
   p.status = status;
+  p.o_store32 = (reinterpret_cast<uintptr_t>(O) & 31u) == 0;
   const size_t smem = 1024 + kTileBytes * (kSlots + kStages) + sizeof(Smem);
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));

@@ -269,3 +269,20 @@ def test_maximum_block_count():
     res = run_gpu(prob)
     qblocks = [0, 1, 2047, 3000, 4094, 4095]
     check_problem(prob, [0], qblocks, res)
+
+
+def test_output_only_16_byte_aligned():
+    """O at a 16-byte but not 32-byte aligned address takes the 16-byte store
+    path and gives the same result as an aligned O."""
+    prob = make_problem("c1", L=2048, hq=2, hkv=1)
+    Q, K, V = prob.Q.to(DEV), prob.K.to(DEV), prob.V.to(DEV)
+    P = xattn_score(Q, K, prob.B, prob.S, prob.causal)
+    _, counts, idx = xattn_select(P, prob.tau.tolist(), prob.causal)
+    ref = xattn_sparse_attn(Q, K, V, counts, idx, prob.B, prob.causal)
+    flat = torch.empty(Q.numel() + 16, device=DEV, dtype=Q.dtype)
+    out = flat[8:8 + Q.numel()].view(Q.shape)   # 8 bf16 = 16 bytes past a 256-byte base
+    assert out.data_ptr() % 32 == 16
+    xattn_sparse_attn(Q, K, V, counts, idx, prob.B, prob.causal, out=out)
+    torch.cuda.synchronize()
+    assert xattn_get_device_status() == 0
+    assert torch.equal(out, ref)
