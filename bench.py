@@ -40,10 +40,10 @@ WORKLOAD = "c2"   # the 128K Llama-shaped layer the metric is quoted on
 # KV groups, every query block); traffic grows with the number of heads, so the
 # figures are scaled by 32 / 8 to a full call. Summaries: profiles/.
 TRAFFIC_BYTES = {
-    # score_tc 358.13 MB read + 120.59 MB written; score_reduce 134.38 + 19.69 MB
-    ("c2", "score"): 4 * (358.13 + 120.59 + 134.38 + 19.69) * 1e6,
-    # attn_tc 841.86 MB read + 237.50 MB written (sched_kernel: 1.12 MB)
-    ("c2", "sparse_attn"): 4 * (841.86 + 237.50 + 1.12) * 1e6,
+    # score_tc 353.85 MB read + 121.10 MB written; score_reduce 134.37 + 18.82 MB
+    ("c2", "score"): 4 * (353.85 + 121.10 + 134.37 + 18.82) * 1e6,
+    # attn_tc 863.80 MB read + 238.14 MB written (sched_kernel: 1.12 MB)
+    ("c2", "sparse_attn"): 4 * (863.80 + 238.14 + 1.12) * 1e6,
 }
 
 
