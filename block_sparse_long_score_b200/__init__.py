@@ -6,14 +6,16 @@ Three steps, each one call into the C-ABI library ``libxattn.so``:
 attention over the selected blocks). The pages' ablation variants run
 through the same kernels: ``xattn_score_pattern`` (diagonal or random
 sampling) and ``xattn_select_topk`` / ``xattn_select_topratio`` (fixed
-budgets). The library loads on first use and the calls raise if it is
-missing.
+budgets). ``xattn_prefill_host`` runs the whole step on host tensors with the
+host<->device copies overlapped with the compute. The library loads on first
+use and the calls raise if it is missing.
 """
 from .xattn import (  # noqa: F401
     XattnError, xattn_score, xattn_select, xattn_sparse_attn, xattn_score_workspace_bytes,
     xattn_attn_workspace_bytes, xattn_get_device_status, xattn_strerror, make_shape,
     library_path, EXPORTED_SYMBOLS, xattn_sparse_attn_noalloc, xattn_score_pattern,
     xattn_select_topk, xattn_select_topratio, antidiagonal_perm, diagonal_perm,
-    xattn_score_select, xattn_selftest_timeout,
+    xattn_score_select, xattn_selftest_timeout, xattn_prefill_host,
+    xattn_prefill_host_workspace_bytes,
 )
 from .pipeline import prefill_attention  # noqa: F401

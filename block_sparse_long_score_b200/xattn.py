@@ -22,6 +22,7 @@ __all__ = [
     "EXPORTED_SYMBOLS", "xattn_sparse_attn_noalloc", "NOALLOC_MAX_UNITS",
     "xattn_score_pattern", "xattn_select_topk", "xattn_select_topratio",
     "antidiagonal_perm", "diagonal_perm", "xattn_score_select", "xattn_selftest_timeout",
+    "xattn_prefill_host_workspace_bytes", "xattn_prefill_host",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -33,7 +34,7 @@ EXPORTED_SYMBOLS = (
     "xattn_attn_workspace_bytes", "xattn_sparse_attn", "xattn_get_device_status",
     "xattn_strerror", "xattn_sparse_attn_noalloc", "xattn_score_pattern",
     "xattn_select_topk", "xattn_select_topratio", "xattn_score_select",
-    "xattn_selftest_timeout",
+    "xattn_selftest_timeout", "xattn_prefill_host_workspace_bytes", "xattn_prefill_host",
 )
 # batch * hq * (L / B) limit of xattn_sparse_attn_noalloc (XATTN_NOALLOC_MAX_UNITS)
 NOALLOC_MAX_UNITS = 1 << 18
@@ -91,6 +92,11 @@ def _lib() -> ctypes.CDLL:
         lib.xattn_sparse_attn.restype = i32
         lib.xattn_sparse_attn_noalloc.argtypes = [vp, vp, vp, sp, vp, vp, vp, vp, vp]
         lib.xattn_sparse_attn_noalloc.restype = i32
+        lib.xattn_prefill_host_workspace_bytes.argtypes = [sp, i32]
+        lib.xattn_prefill_host_workspace_bytes.restype = sz
+        lib.xattn_prefill_host.argtypes = [vp, vp, vp, sp, ctypes.POINTER(ctypes.c_float), vp,
+                                           vp, i32, vp, sz, vp]
+        lib.xattn_prefill_host.restype = i32
         lib.xattn_selftest_timeout.argtypes = [vp]
         lib.xattn_selftest_timeout.restype = i32
         lib.xattn_get_device_status.argtypes = [vp]
@@ -357,6 +363,58 @@ def xattn_sparse_attn_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                                           _stream(Q.device))
     _raise("xattn_sparse_attn_noalloc", rc)
     return out
+
+
+def xattn_prefill_host_workspace_bytes(shape: _Shape, kv_heads_per_chunk: int = 0) -> int:
+    return int(_lib().xattn_prefill_host_workspace_bytes(ctypes.byref(shape),
+                                                         int(kv_heads_per_chunk)))
+
+
+def _check_any(t: torch.Tensor, name: str, dtype=None) -> None:
+    """Layout and type check of a tensor that may live in host or device memory."""
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def xattn_prefill_host(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, B: int, S: int,
+                       causal: bool, tau: Sequence[float], out: Optional[torch.Tensor] = None,
+                       lse: Optional[torch.Tensor] | bool = None, kv_heads_per_chunk: int = 0,
+                       workspace: Optional[torch.Tensor] = None, device=None):
+    """The whole prefill step (score + select with threshold tau, then sparse
+    attention) on Q, K, V in host memory -- pinned for the copies to overlap
+    the compute -- with O (and lse) written to host memory. Runs on the current
+    stream of ``device`` (the current CUDA device by default); synchronise it
+    before reading ``out``. Returns O, or (O, lse) if lse is True or a tensor."""
+    _check_any(Q, "Q")
+    _check_any(K, "K", Q.dtype)
+    _check_any(V, "V", Q.dtype)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None \
+        else torch.device(device)
+    shape = _shape_of(Q, K, B, S, causal)
+    if out is None:
+        out = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=not Q.is_cuda,
+                          device=Q.device)
+    _check_any(out, "O", Q.dtype)
+    want_lse = lse is not None and lse is not False
+    if lse is True:
+        lse = torch.empty(Q.shape[:3], dtype=torch.float32, pin_memory=not Q.is_cuda,
+                          device=Q.device)
+    if want_lse:
+        _check_any(lse, "lse", torch.float32)
+    taus = _per_head(tau, shape.hq, "tau", float)
+    tarr = (ctypes.c_float * shape.hq)(*taus)
+    need = xattn_prefill_host_workspace_bytes(shape, kv_heads_per_chunk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=dev, dtype=torch.uint8)
+    _check(workspace, "workspace")
+    rc = _lib().xattn_prefill_host(Q.data_ptr(), K.data_ptr(), V.data_ptr(), ctypes.byref(shape),
+                                   tarr, out.data_ptr(), lse.data_ptr() if want_lse else None,
+                                   int(kv_heads_per_chunk), workspace.data_ptr(),
+                                   workspace.numel() * workspace.element_size(), _stream(dev))
+    _raise("xattn_prefill_host", rc)
+    return (out, lse) if want_lse else out
 
 
 def xattn_selftest_timeout(device=None) -> None:

@@ -229,6 +229,51 @@ int xattn_sparse_attn_noalloc(const void* Q, const void* K, const void* V,
                               const int32_t* idx, void* O, float* lse, void* stream);
 
 /*
+ * Workspace bytes of xattn_prefill_host for a shape and a chunk size (see
+ * below). Returns 0 for an invalid shape or chunk size.
+ */
+size_t xattn_prefill_host_workspace_bytes(const xattn_shape* shape, int kv_heads_per_chunk);
+
+/*
+ * The whole prefill step of one layer -- xattn_score_select (threshold tau),
+ * then xattn_sparse_attn -- on Q, K, V held in HOST memory, writing O (and
+ * lse) back to host memory. Results are bit-identical to those two calls on
+ * device copies of the same tensors. This entry point has no counterpart in
+ * the paper: it is the step as a host program sees it, with the
+ * host<->device copies overlapped with the compute.
+ * Every step of the method is independent across KV heads, so the call cuts
+ * the layer into chunks of kv_heads_per_chunk KV heads (with their hq/hkv
+ * query heads each) per batch entry; 0 means 1, and a last chunk of a batch
+ * entry may be smaller when hkv is not a multiple. Each chunk goes through a
+ * ring of two device slots: copy in on one internal stream, compute on
+ * `stream`, copy out on a second internal stream, so chunk c+1 is copied in
+ * and chunk c-1 copied out while chunk c is computed.
+ * Q, K, V: [batch, heads, L, d] contiguous, as for xattn_sparse_attn, in host
+ *          memory (page-locked, e.g. from cudaHostAlloc, for the copies to
+ *          overlap; pageable memory gives the same results more slowly) or
+ *          device memory. Not modified.
+ * tau:     HOST pointer to hq floats in (0, 1], as for xattn_select.
+ * O:       out, [batch, hq, L, d] of the same type, host or device memory.
+ * lse:     out, optional (may be NULL), fp32 [batch, hq, L], as for
+ *          xattn_sparse_attn.
+ * ws / ws_bytes: DEVICE workspace of at least
+ *          xattn_prefill_host_workspace_bytes(shape, kv_heads_per_chunk)
+ *          bytes, 256-byte aligned; it holds the two slots and the scratch of
+ *          both steps (WORKSPACE otherwise).
+ * Ordering: the call is asynchronous on `stream` like every other call: the
+ * copies start after the work queued on `stream` before the call, and work
+ * queued on `stream` after it starts once O and lse are in place. The host
+ * buffers must stay valid and unchanged until then. The call creates, and
+ * releases, its two copy streams and its events on each call.
+ * Errors: INVALID_ARG (NULL pointer, bad shape or tau, kv_heads_per_chunk < 0
+ * or > hkv), UNSUPPORTED and CUDA as for the two steps, WORKSPACE. A failure
+ * part-way through leaves O partly written.
+ */
+int xattn_prefill_host(const void* Q, const void* K, const void* V, const xattn_shape* shape,
+                       const float* tau, void* O, float* lse, int kv_heads_per_chunk, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's status
  * word. Returns XATTN_OK, XATTN_ERR_TIMEOUT if a kernel gave up a bounded
  * wait since the last call, or XATTN_ERR_CUDA if the stream reports an error.

@@ -146,3 +146,47 @@ def test_score_select_host_checks(lib):
     assert f(FAKE, FAKE, ctypes.byref(s), good, None, FAKE, FAKE, FAKE, FAKE, 16, None) == -4
     odd = ctypes.c_void_p(0x10008)
     assert f(odd, FAKE, ctypes.byref(s), good, None, FAKE, FAKE, FAKE, FAKE, 1 << 40, None) == -1
+
+
+def _r256(x):
+    return (x + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("ck", [0, 1, 3, 8])
+def test_prefill_host_workspace_size(lib, ck):
+    """Two slots of one chunk's Q, K, V, O and lse, plus one chunk's selection
+    outputs and the two steps' workspaces."""
+    s = X.make_shape(1, 32, 8, 131072, 128, 128, 16, True, "bf16")
+    c = max(ck, 1)
+    hq_c, L, NB = 4 * c, 131072, 1024
+    row = L * 128 * 2
+    cs = X.make_shape(1, hq_c, c, L, 128, 128, 16, True, "bf16")
+    slot = _r256(hq_c * row) * 2 + _r256(c * row) * 2 + _r256(hq_c * L * 4)
+    want = 2 * slot + _r256(hq_c * NB * 32 * 4) + _r256(hq_c * NB * 4) + \
+        _r256(hq_c * NB * NB * 4) + _r256(X.xattn_score_workspace_bytes(cs)) + \
+        _r256(X.xattn_attn_workspace_bytes(cs))
+    assert X.xattn_prefill_host_workspace_bytes(s, ck) == want
+
+
+def test_prefill_host_checks(lib):
+    s = X.make_shape(2, 4, 2, 1024, 128, 128, 8, True, "bf16")
+    good = (ctypes.c_float * 4)(0.9, 0.9, 0.9, 0.9)
+    bad = (ctypes.c_float * 4)(0.9, 0.0, 0.9, 0.9)
+    f = lib.xattn_prefill_host
+    big = 1 << 40
+    assert X.xattn_prefill_host_workspace_bytes(s, -1) == 0
+    assert X.xattn_prefill_host_workspace_bytes(s, 3) == 0      # more than hkv
+    assert f(None, FAKE, FAKE, ctypes.byref(s), good, FAKE, None, 0, FAKE, big, None) == -1
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(s), good, None, None, 0, FAKE, big, None) == -1
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(s), None, FAKE, None, 0, FAKE, big, None) == -1
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(s), bad, FAKE, None, 0, FAKE, big, None) == -1
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(s), good, FAKE, None, -1, FAKE, big, None) == -1
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(s), good, FAKE, None, 3, FAKE, big, None) == -1
+    assert f(FAKE, FAKE, FAKE, None, good, FAKE, None, 0, FAKE, big, None) == -1
+    need = X.xattn_prefill_host_workspace_bytes(s, 0)
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(s), good, FAKE, None, 0, None, big, None) == -4
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(s), good, FAKE, None, 0, FAKE, need - 1, None) == -4
+    odd = ctypes.c_void_p(0x10080)                               # not 256-byte aligned
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(s), good, FAKE, None, 0, odd, big, None) == -4
+    wide = X.make_shape(1, 4, 2, 1024, 64, 128, 8, True, "bf16")  # bf16 needs d = 128
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(wide), good, FAKE, None, 0, FAKE, big, None) == -2
