@@ -33,6 +33,13 @@ Readings where the pages are silent or garbled:
 * tau >= 1, or a cumulative sum that never reaches tau, selects every allowed
   block.
 * GQA: query head h reads KV head h // (Hq / Hkv).
+* A sequence whose length L is not a multiple of B (Algorithm 1 only walks
+  floor(L/B) whole blocks) ends in a shorter last block: NB = ceil(L/B), and
+  the last query / key block holds the L - (NB-1)B remaining tokens. L must be
+  a multiple of S, so every reshaped row and column is whole. The softmax rows
+  run over the L/S reshaped columns that exist, and P[b, j] divides by the
+  number of reshaped rows block b actually has (r for a whole block), so every
+  row of P still sums to 1.
 
 Everything runs in float64. bf16 and fp32 inputs convert to float64 exactly.
 Matrix products go through numpy's matmul (a library primitive); everything
@@ -182,8 +189,8 @@ def block_probs_head(q: np.ndarray, k: np.ndarray, B: int, S: int, causal: bool,
     reshape_queries); the default is the antidiagonal.
     """
     L, d = q.shape
-    assert L % B == 0 and B % S == 0
-    NB, r = L // B, B // S
+    assert L % S == 0 and B % S == 0
+    NB, r, R = -(-L // B), B // S, L // S
     scale = 1.0 / math.sqrt(d * S)
     Qr = reshape_queries(q, S, perm)
     Kr = reshape_keys(k, S)
@@ -192,15 +199,25 @@ def block_probs_head(q: np.ndarray, k: np.ndarray, B: int, S: int, causal: bool,
     per_chunk = max(1, chunk_rows // r)
     for i0 in range(0, len(blocks), per_chunk):
         group = blocks[i0:i0 + per_chunk]
-        rows = np.concatenate([np.arange(b * r, (b + 1) * r) for b in group])
-        ncols = (max(group) + 1) * r if causal else Kr.shape[0]
+        # reshaped rows of block b: [b*r, min((b+1)*r, R)); the last block may be short
+        spans = [(b * r, min((b + 1) * r, R)) for b in group]
+        rows = np.concatenate([np.arange(a, e) for a, e in spans])
+        ncols = min((max(group) + 1) * r, R) if causal else R
         x = (Qr[rows] @ Kr[:ncols].T) * scale
-        for gi, b in enumerate(group):
-            xb = x[gi * r:(gi + 1) * r]
-            A = approx_attention_rows(xb, b * r, causal)
+        o = 0
+        for (a, e), b in zip(spans, group):
+            rb = e - a
+            xb = x[o:o + rb]
+            o += rb
+            A = approx_attention_rows(xb, a, causal)
             nj = b + 1 if causal else NB
-            # sum each r x r sub-block, then divide by r
-            blk = A[:, : nj * r].reshape(r, nj, r).sum(axis=(0, 2)) / r
+            # columns of key block j: [j*r, min((j+1)*r, R)); pad the missing
+            # columns of a short last block with zeros, sum each sub-block,
+            # then divide by the block's number of rows
+            Ap = np.zeros((rb, nj * r))
+            w = min(nj * r, A.shape[1])
+            Ap[:, :w] = A[:, :w]
+            blk = Ap.reshape(rb, nj, r).sum(axis=(0, 2)) / rb
             P[b, :] = 0.0
             P[b, :nj] = blk
     return P
@@ -216,7 +233,7 @@ def block_probs(Q, K, B: int, S: int, causal: bool, heads: Sequence[int] | None 
     Qf, Kf = to_f64(Q), to_f64(K)
     b_, hq, L, d = Qf.shape
     hkv = Kf.shape[1]
-    NB = L // B
+    NB = -(-L // B)
     out = np.full((b_, hq, NB, NB), np.nan)
     hs = range(hq) if heads is None else heads
     for bb in range(b_):
@@ -369,18 +386,18 @@ def sparse_attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, B: int,
     with no visible key gets O = 0 and lse = -inf.
     """
     L, d = q.shape
-    NB = L // B
+    NB = -(-L // B)
     O = np.full((L, v.shape[1]), np.nan)
     lse = np.full(L, np.nan)
     blocks = range(NB) if q_blocks is None else q_blocks
     for b in blocks:
         kb = np.asarray(block_lists[b], dtype=np.int64)
-        qi = np.arange(b * B, (b + 1) * B)
+        qi = np.arange(b * B, min((b + 1) * B, L))   # the last block may be short
         if kb.size == 0:
             O[qi] = 0.0
             lse[qi] = -np.inf
             continue
-        keys = (kb[:, None] * B + np.arange(B)[None, :]).reshape(-1)
+        keys = np.concatenate([np.arange(j * B, min((j + 1) * B, L)) for j in kb])
         logits = (q[qi] @ k[keys].T) / math.sqrt(d)
         if causal:
             logits[keys[None, :] > qi[:, None]] = -np.inf
@@ -407,7 +424,7 @@ def sparse_attention(Q, K, V, B: int, causal: bool, lists: dict,
     O = np.full(Qf.shape[:3] + (Vf.shape[3],), np.nan)
     lse = np.full((b_, hq, L), np.nan)
     hs = range(hq) if heads is None else heads
-    NB = L // B
+    NB = -(-L // B)
     for bb in range(b_):
         for h in hs:
             kv = kv_head(h, hq, hkv)

@@ -437,3 +437,91 @@ def test_select_topk_and_topratio_rows(causal):
                 dropped = np.setdiff1d(np.arange(n), sel)
                 if len(dropped):
                     assert P[0, h, b, sel].min() >= P[0, h, b, dropped].max()
+
+
+# ------------------------------------------------- short last block (L % B) --
+# A length that is not a multiple of B ends in a shorter last block. These pins
+# check the oracle's reading of that case against facts from outside it.
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("S", [2, 4, 8])
+def test_short_last_block_rows_are_distributions(causal, S):
+    """L = 232 with B = 32: NB = 8 and the last block has 8 tokens. Every row
+    of P, the short one included, still sums to 1 (a divisor of r instead of
+    the block's own row count would give 8/32 on the last row)."""
+    q, k = _rand(232, 16), _rand(232, 16)
+    P = O.block_probs_head(q, k, 32, S, causal)
+    assert P.shape == (8, 8)
+    np.testing.assert_allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    assert (P >= 0).all()
+    if causal:
+        assert np.all(P[np.triu_indices(8, 1)] == 0.0)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_short_last_block_stride_one_is_exact_attention(causal):
+    """S = 1, L = 44, B = 8: the last block has 4 tokens. P[b, j] is the mean
+    over block b's queries of the naive attention mass on block j's keys."""
+    L, B = 44, 8
+    q, k = _rand(L, 4), _rand(L, 4)
+    P = O.block_probs_head(q, k, B, 1, causal)
+    _, probs = O.dense_attention_naive(q, k, np.zeros((L, 1)), causal)
+    NB = 6
+    want = np.zeros((NB, NB))
+    for i in range(L):
+        for j in range(L):
+            want[i // B, j // B] += probs[i, j]
+    for b in range(NB):
+        want[b] /= min(B, L - b * B)
+    np.testing.assert_allclose(P, want, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("S", [2, 4])
+def test_short_last_block_causal_rows_ignore_the_tail(S):
+    """Causal: the rows of the whole blocks see no token after their block, so
+    they equal the P of the sequence cut after its last whole block."""
+    q, k = _rand(232, 8), _rand(232, 8)
+    P = O.block_probs_head(q, k, 32, S, True)
+    Pc = O.block_probs_head(q[:224], k[:224], 32, S, True)
+    np.testing.assert_allclose(P[:7, :7], Pc, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_short_last_block_dense_mask_is_naive_attention(causal):
+    """L = 28, B = 8 (last block: 4 tokens): attention over every allowed
+    block equals the naive triple loop over the 28 keys."""
+    L, B, NB = 28, 8, 4
+    q, k, v = _rand(L, 4), _rand(L, 4), _rand(L, 3)
+    lists = {b: list(range(b + 1 if causal else NB)) for b in range(NB)}
+    Os, lse = O.sparse_attention_head(q, k, v, B, causal, lists)
+    On, _ = O.dense_attention_naive(q, k, v, causal)
+    np.testing.assert_allclose(Os, On, rtol=0, atol=1e-12)
+    raw = O.dense_scores(q, k) / math.sqrt(4)
+    for i in range(L):
+        n = i + 1 if causal else L
+        want = math.log(math.fsum(math.exp(x) for x in raw[i, :n]))
+        assert abs(lse[i] - want) < 1e-12
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_short_last_block_lists_match_filtered_naive_attention(causal):
+    L, B, NB = 60, 8, 8
+    q, k, v = _rand(L, 4), _rand(L, 4), _rand(L, 5)
+    lists = {}
+    for b in range(NB):
+        n = b + 1 if causal else NB
+        lists[b] = sorted({0} | {j for j in range(n) if rng.random() < 0.5})
+    Os, _ = O.sparse_attention_head(q, k, v, B, causal, lists)
+    On, _ = O.dense_attention_naive(q, k, v, causal,
+                                    allowed=lambda i, j: (j // B) in lists[i // B])
+    np.testing.assert_allclose(Os, On, rtol=0, atol=1e-12)
+
+
+def test_short_last_block_batched_shapes():
+    """The batched wrappers size P and O by ceil(L / B) blocks."""
+    Q, K, V = _rand(1, 2, 40, 4), _rand(1, 1, 40, 4), _rand(1, 1, 40, 4)
+    P = O.block_probs(Q, K, 16, 4, True)
+    assert P.shape == (1, 2, 3, 3)
+    _, lists = O.select_blocks(P, [0.9, 1.0], True)
+    Os, lse = O.sparse_attention(Q, K, V, 16, True, lists)
+    assert Os.shape == (1, 2, 40, 4) and np.isfinite(Os).all() and np.isfinite(lse).all()
