@@ -63,10 +63,12 @@ int check_shape(const xattn_shape* sh, Dims* D) {
   if (s.batch < 1 || s.hq < 1 || s.hkv < 1 || s.L < 1 || s.d < 1 || s.B < 1 || s.S < 1)
     return XATTN_ERR_INVALID_ARG;
   if (s.hq % s.hkv != 0) return XATTN_ERR_INVALID_ARG;
-  if (s.L % s.B != 0 || s.B % s.S != 0) return XATTN_ERR_INVALID_ARG;
+  // L need not be a multiple of B (the last block is then shorter), but it
+  // must be a multiple of S so that every reshaped row and column is whole
+  if (s.L % s.S != 0 || s.B % s.S != 0) return XATTN_ERR_INVALID_ARG;
   if (s.dtype != XATTN_F32 && s.dtype != XATTN_BF16) return XATTN_ERR_INVALID_ARG;
   if (s.hq > XATTN_MAX_HEADS) return XATTN_ERR_UNSUPPORTED;
-  const int NB = s.L / s.B;
+  const int NB = (s.L + s.B - 1) / s.B;
   if (NB > XATTN_MAX_BLOCKS) return XATTN_ERR_UNSUPPORTED;
   if (static_cast<long long>(s.batch) * s.hq * s.L > (1ll << 31) - 1) return XATTN_ERR_UNSUPPORTED;
   if (static_cast<long long>(s.batch) * s.hq * NB > (1ll << 24)) return XATTN_ERR_UNSUPPORTED;
@@ -88,6 +90,7 @@ int check_shape(const xattn_shape* sh, Dims* D) {
   D->NB = NB;
   D->r = s.B / s.S;
   D->R = s.L / s.S;
+  D->tail = s.L - (NB - 1) * s.B;
   D->group = s.hq / s.hkv;
   return XATTN_OK;
 }

@@ -47,9 +47,10 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int kb = list[jj];
     if (D.causal && kb > qb) break;  // ascending list: the rest is above the diagonal
     if (kb < 0 || kb >= D.NB) continue;
-    for (int k0 = kb * D.B; k0 < (kb + 1) * D.B; k0 += 32) {
+    const int kend = min((kb + 1) * D.B, D.L);  // a short last block ends at L
+    for (int k0 = kb * D.B; k0 < kend; k0 += 32) {
       const int key = k0 + lane;
-      const bool valid = key < (kb + 1) * D.B && !(D.causal && key > q);
+      const bool valid = key < kend && !(D.causal && key > q);
       float sc = -INFINITY;
       if (valid) {
         const float* kr = Kh + static_cast<size_t>(key) * d;

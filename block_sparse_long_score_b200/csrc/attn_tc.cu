@@ -62,6 +62,7 @@ static_assert(128 * (kCtrlRegs + kSoftmaxRegs + kEpiRegs) <= kThreads * kLaunchR
 
 struct Params {
   int L, NB, hq, hkv, group, causal, units;
+  int tail;          // tokens of the last block (B unless the length is ragged)
   float scale_log2;  // log2(e) / sqrt(d)
   const int32_t* counts;
   const int32_t* idx;
@@ -95,7 +96,10 @@ __device__ __forceinline__ int entry_unit(unsigned long long e) {
 __device__ __forceinline__ int entry_count(unsigned long long e) {
   return static_cast<int>((e >> 32) & 0xFFFFull);
 }
-__device__ __forceinline__ bool entry_diag(unsigned long long e) { return (e >> 48) & 1ull; }
+// The unit's last listed block needs a column mask: the diagonal block
+// (causal: keys after the query), or the short last block (non-causal: keys
+// at or past L).
+__device__ __forceinline__ bool entry_masked(unsigned long long e) { return (e >> 48) & 1ull; }
 
 // Walks the blocks of this CTA's units in order, skipping units with no block.
 // The next unit's entry is always one load ahead; the producer (kList) also
@@ -387,13 +391,15 @@ __device__ __forceinline__ void softmax_role(const Params& p, Smem* sm, uint32_t
     if (n <= 0) continue;                   // the epilogue warpgroup writes it
     const uint32_t ob = u & 1;
     const uint32_t tO = tmem + lane_addr + kColO + ob * kD;
-    // a causal list is ascending and ends at most at qb: only its last
-    // block can be the diagonal one (flagged in the order entry)
-    const bool last_is_diag = entry_diag(e);
+    // lists are ascending: only the last block can be the diagonal one
+    // (causal, ends at most at qb) or the short last one (flagged in the
+    // order entry). Keep columns <= lim of that block.
+    const bool last_masked = entry_masked(e);
+    const int lim = p.causal ? row : p.tail - 1;
     float m_run = -INFINITY;  // running max of scaled logits (log2 units)
     float l_run = 0.f;
     for (int j = 0; j < n; ++j, ++g) {
-      const bool diag = last_is_diag && j == n - 1;
+      const bool masked = last_masked && j == n - 1;
       const uint32_t sb = g & 1;
       const uint32_t tS = tmem + lane_addr + sb * kBlk;
       if (!warp_wait(&sm->s_full[sb], (g >> 1) & 1, abort)) return;
@@ -402,12 +408,12 @@ __device__ __forceinline__ void softmax_role(const Params& p, Smem* sm, uint32_t
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sv[c]);
       tmem_ld_wait();
-      if (diag) {
+      if (masked) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (c * 32 + i > row) sv[c][i] = __float_as_uint(-INFINITY);
+            if (c * 32 + i > lim) sv[c][i] = __float_as_uint(-INFINITY);
       }
       float mx;
       {
@@ -510,7 +516,10 @@ __device__ __forceinline__ void epilogue_role(const Params& p, Smem* sm, uint32_
     const int n = entry_count(e);
     const size_t orow = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qb) * kBlk + row;
     __nv_bfloat16* optr = p.O + orow * kD;
+    // rows past L in a short last block belong to no query: nothing is stored
+    const bool row_valid = qb < p.NB - 1 || row < p.tail;
     if (n <= 0) {
+      if (!row_valid) continue;
       const uint4 z = make_uint4(0, 0, 0, 0);
       for (int c = 0; c < kD / 8; ++c) reinterpret_cast<uint4*>(optr)[c] = z;
       if (p.lse) p.lse[orow] = -INFINITY;
@@ -528,8 +537,9 @@ __device__ __forceinline__ void epilogue_role(const Params& p, Smem* sm, uint32_
 #pragma unroll 1
     for (int c = 0; c < kD / 32; ++c) {
       uint32_t v[32];
-      tmem_ld32(tO + c * 32, v);
+      tmem_ld32(tO + c * 32, v);  // warp-collective: every lane loads
       tmem_ld_wait();
+      if (!row_valid) continue;
       uint32_t w[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i)
@@ -545,7 +555,7 @@ __device__ __forceinline__ void epilogue_role(const Params& p, Smem* sm, uint32_
           dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
       }
     }
-    if (p.lse) p.lse[orow] = (m_run + lg2(l_run)) * 0.69314718055994531f;
+    if (p.lse && row_valid) p.lse[orow] = (m_run + lg2(l_run)) * 0.69314718055994531f;
     tc_fence_before();
     mbar_arrive(&sm->o_empty[ob]);
     ++u;
@@ -641,6 +651,7 @@ cudaError_t launch_attn_tc(const Dims& D, const CUtensorMap& tmQ, const CUtensor
   p.group = D.group;
   p.causal = D.causal;
   p.units = D.batch * D.hq * D.NB;
+  p.tail = D.tail;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(double(D.d)));
   p.counts = counts;
   p.idx = idx;

@@ -16,7 +16,8 @@ constexpr int kStatusTimeout = 1;
 
 struct Dims {
   int batch, hq, hkv, L, d, B, S, causal, dtype;
-  int NB, r, R, group;  // L/B, B/S, L/S, hq/hkv
+  int NB, r, R, group;  // ceil(L/B), B/S, L/S, hq/hkv
+  int tail;             // tokens of the last block: L - (NB-1)*B (B when B divides L)
 };
 
 // Partial log-sum-exp workspace of the scoring step.

@@ -5,9 +5,10 @@
 // produce the same P bit for bit.
 //
 // Input: for every reshaped query row rho and allowed key block j, the partial
-// L[rho, j] = log2 sum_{c in block j} 2^(x[rho, c] log2 e). For query block b:
+// L[rho, j] = log2 sum_{c in block j} 2^(x[rho, c] log2 e). For query block b
+// with r_b reshaped rows (r, or fewer for a short last block):
 //   LSE[rho]  = log2 sum_j 2^L[rho, j]                (row normaliser)
-//   P[b, j]   = (1/r) sum_{rho in block b} 2^(L[rho, j] - LSE[rho])
+//   P[b, j]   = (1/r_b) sum_{rho in block b} 2^(L[rho, j] - LSE[rho])
 // and P[b, j] = 0 for the causally masked j > b.
 #pragma once
 
@@ -17,17 +18,25 @@
 namespace xattn {
 namespace red {
 
-// Fills row_off[t] and lse[t] (t < r) for query block b; every thread of the
-// CTA takes part, and the function ends with __syncthreads.
+// Number of reshaped rows of query block b: r, or fewer for a short last block.
+__device__ __forceinline__ int block_rows(int b, int r, int R) {
+  const int left = R - b * r;
+  return left < r ? left : r;
+}
+
+// Fills row_off[t] and lse[t] (t < rb, the block's reshaped rows) for query
+// block b; every thread of the CTA takes part, and the function ends with
+// __syncthreads.
 __device__ __forceinline__ void block_row_lse(const float* __restrict__ base, int b, int NB, int r,
-                                              int nj, bool causal, float* lse, size_t* row_off) {
+                                              int rb, int nj, bool causal, float* lse,
+                                              size_t* row_off) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int nwarps = blockDim.x / 32;
-  for (int t = threadIdx.x; t < r; t += blockDim.x)
+  for (int t = threadIdx.x; t < rb; t += blockDim.x)
     row_off[t] = part_row_offset(b * r + t, r, NB, causal);
   __syncthreads();
   // row log-sum-exp: online (max, sum) over 8 loads in flight per lane
-  for (int t = warp; t < r; t += nwarps) {
+  for (int t = warp; t < rb; t += nwarps) {
     const float* row = base + row_off[t];
     float m = -INFINITY, s = 0.f;
     for (int j0 = 0; j0 < nj; j0 += 8 * 32) {
@@ -63,7 +72,8 @@ __device__ __forceinline__ void block_row_lse(const float* __restrict__ base, in
   __syncthreads();
 }
 
-// P[b, j] for an allowed block j < nj; r loads in flight per thread.
+// P[b, j] for an allowed block j < nj over the block's r (= r_b) rows; r loads
+// in flight per thread.
 __device__ __forceinline__ float block_prob(const float* __restrict__ base, const size_t* row_off,
                                             const float* lse, int r, int j, float inv_r) {
   float acc = 0.f;

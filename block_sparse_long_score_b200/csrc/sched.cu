@@ -11,7 +11,9 @@
 //   bits  0..31  unit index (bh * NB + query block)
 //   bits 32..47  effective block count: causal lists drop trailing blocks above
 //                the diagonal (lists are ascending)
-//   bit  48      the last listed block is the diagonal block (causal)
+//   bit  48      the last listed block needs a column mask: it is the diagonal
+//                block (causal), or the short last block of a sequence whose
+//                length B does not divide (non-causal)
 #include "common.cuh"
 
 namespace xattn {
@@ -19,11 +21,12 @@ namespace {
 
 constexpr int kThreads = 1024;
 
-// Effective block count and diagonal flag of units u, u + kThreads, ...
+// Effective block count and mask flag (bit 48) of units u, u + kThreads, ...
 // (8 of them): causal lists drop trailing blocks above the diagonal.
 __device__ __forceinline__ void unit_info8(const int32_t* __restrict__ counts,
                                            const int32_t* __restrict__ idx, int u, int units,
-                                           int NB, int causal, int (&n)[8], bool (&diag)[8]) {
+                                           int NB, int causal, int ragged, int (&n)[8],
+                                           bool (&diag)[8]) {
   int c[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
@@ -49,6 +52,14 @@ __device__ __forceinline__ void unit_info8(const int32_t* __restrict__ counts,
       }
       diag[q] = uu < units && c[q] > 0 && last[q] == qb;
     }
+  } else if (ragged) {
+    // non-causal with a short last block: lists are ascending, so block NB-1
+    // can only be a list's last entry
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int uu = u + q * kThreads;
+      diag[q] = uu < units && c[q] > 0 && idx[static_cast<size_t>(uu) * NB + c[q] - 1] == NB - 1;
+    }
   } else {
 #pragma unroll
     for (int q = 0; q < 8; ++q) diag[q] = false;
@@ -59,7 +70,7 @@ __device__ __forceinline__ void unit_info8(const int32_t* __restrict__ counts,
 
 __global__ void __launch_bounds__(kThreads)
     sched_kernel(const int32_t* __restrict__ counts, const int32_t* __restrict__ idx, int units,
-                 int NB, int causal, unsigned long long* __restrict__ order) {
+                 int NB, int causal, int ragged, unsigned long long* __restrict__ order) {
   extern __shared__ int hist[];  // NB + 1 bins, bin = NB - count
   const int nbins = NB + 1;
   for (int i = threadIdx.x; i < nbins; i += kThreads) hist[i] = 0;
@@ -68,7 +79,7 @@ __global__ void __launch_bounds__(kThreads)
   for (int u0 = 0; u0 < units; u0 += 8 * kThreads) {
     int n[8];
     bool diag[8];
-    unit_info8(counts, idx, u0 + threadIdx.x, units, NB, causal, n, diag);
+    unit_info8(counts, idx, u0 + threadIdx.x, units, NB, causal, ragged, n, diag);
 #pragma unroll
     for (int q = 0; q < 8; ++q)
       if (u0 + threadIdx.x + q * kThreads < units) atomicAdd(&hist[NB - n[q]], 1);
@@ -111,7 +122,7 @@ __global__ void __launch_bounds__(kThreads)
   for (int u0 = 0; u0 < units; u0 += 8 * kThreads) {
     int n[8];
     bool diag[8];
-    unit_info8(counts, idx, u0 + threadIdx.x, units, NB, causal, n, diag);
+    unit_info8(counts, idx, u0 + threadIdx.x, units, NB, causal, ragged, n, diag);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const int u = u0 + threadIdx.x + q * kThreads;
@@ -130,7 +141,8 @@ cudaError_t launch_sched(const Dims& D, const int32_t* counts, const int32_t* id
                          unsigned long long* order, cudaStream_t st) {
   const int units = D.batch * D.hq * D.NB;
   const size_t smem = static_cast<size_t>(D.NB + 1) * sizeof(int);
-  sched_kernel<<<1, kThreads, smem, st>>>(counts, idx, units, D.NB, D.causal, order);
+  sched_kernel<<<1, kThreads, smem, st>>>(counts, idx, units, D.NB, D.causal,
+                                          D.tail != D.B ? 1 : 0, order);
   return cudaGetLastError();
 }
 

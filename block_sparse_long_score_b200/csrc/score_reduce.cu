@@ -5,7 +5,8 @@
 // Input: for every reshaped query row rho and allowed key block j, the partial
 // L[rho, j] = log2 sum_{c in block j} 2^(x[rho, c] log2 e). Per query block b:
 //   LSE[rho]  = log2 sum_j 2^L[rho, j]                (row normaliser)
-//   P[b, j]   = (1/r) sum_{rho in block b} 2^(L[rho, j] - LSE[rho])
+//   P[b, j]   = (1/r_b) sum_{rho in block b} 2^(L[rho, j] - LSE[rho])
+// (r_b = r reshaped rows, or fewer for a short last block)
 // and P[b, j] = 0 for the causally masked j > b. Memory-bound: each partial is
 // read twice (the second read hits L1/L2), P is written once, coalesced.
 #include "reduce_core.cuh"
@@ -25,11 +26,12 @@ __global__ void __launch_bounds__(kThreads)
   const int bh = blockIdx.y;
   const int nj = causal ? b + 1 : NB;
   const float* base = part + static_cast<size_t>(bh) * part_head_elems(NB, r, R, causal != 0);
-  red::block_row_lse(base, b, NB, r, nj, causal != 0, lse, row_off);
+  const int rb = red::block_rows(b, r, R);
+  red::block_row_lse(base, b, NB, r, rb, nj, causal != 0, lse, row_off);
   float* out = probs + (static_cast<size_t>(bh) * NB + b) * NB;
-  const float inv_r = 1.0f / static_cast<float>(r);
+  const float inv_r = 1.0f / static_cast<float>(rb);
   for (int j = threadIdx.x; j < NB; j += kThreads)
-    out[j] = j < nj ? red::block_prob(base, row_off, lse, r, j, inv_r) : 0.f;
+    out[j] = j < nj ? red::block_prob(base, row_off, lse, rb, j, inv_r) : 0.f;
 }
 
 }  // namespace

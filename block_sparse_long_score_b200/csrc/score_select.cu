@@ -32,13 +32,14 @@ __global__ void __launch_bounds__(kThreads)
   const int bh = blockIdx.y;
   const int nj = causal ? b + 1 : NB;
   const float* base = part + static_cast<size_t>(bh) * part_head_elems(NB, r, R, causal != 0);
-  red::block_row_lse(base, b, NB, r, nj, causal != 0, lse, row_off);
+  const int rb = red::block_rows(b, r, R);
+  red::block_row_lse(base, b, NB, r, rb, nj, causal != 0, lse, row_off);
 
   const long long row = static_cast<long long>(bh) * NB + b;
   float* out = probs ? probs + row * NB : nullptr;
-  const float inv_r = 1.0f / static_cast<float>(r);
+  const float inv_r = 1.0f / static_cast<float>(rb);
   for (int j = threadIdx.x; j < NB; j += kThreads) {
-    const float pj = j < nj ? red::block_prob(base, row_off, lse, r, j, inv_r) : 0.f;
+    const float pj = j < nj ? red::block_prob(base, row_off, lse, rb, j, inv_r) : 0.f;
     if (out) out[j] = pj;
     if (j < nj) keys[j] = __float_as_uint(pj) & 0x7FFFFFFFu;
   }

@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(kThreads)
     float m = -INFINITY, s = 0.f;
     for (int cc = lane; cc < D.r; cc += 32) {
       const int c = j * D.r + cc;
-      if (D.causal && c > rho) continue;
+      if (c >= D.R || (D.causal && c > rho)) continue;  // short last block / causal
       const float* kr = Kh + static_cast<size_t>(c) * SD;
       float x = 0.f;
       for (int e = 0; e < SD; ++e) x = fmaf(qr[e], kr[e], x);

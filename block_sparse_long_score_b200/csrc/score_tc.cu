@@ -152,7 +152,8 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], int c0, 
       s_run += s * ex2(mb - m_run);
     }
     const int j = c0 / RP;
-    if (((c0 + 32) % RP) == 0) {
+    // the block ends with this chunk, or the row's columns do (a short last block)
+    if (((c0 + 32) % RP) == 0 || c0 + 32 >= R) {
       if (j <= jmax) prow[j] = m_run + lg2(s_run);
       m_run = -INFINITY;
       s_run = 0.f;

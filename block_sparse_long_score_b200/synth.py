@@ -60,7 +60,7 @@ class Problem:
 
     @property
     def NB(self) -> int:
-        return self.L // self.B
+        return -(-self.L // self.B)   # the last block is shorter when B does not divide L
 
 
 # The five workloads. "S" is a list for the stride sweep of the video layer.

@@ -167,14 +167,15 @@ def xattn_score(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal: bool,
                 probs: Optional[torch.Tensor] = None,
                 workspace: Optional[torch.Tensor] = None,
                 perm: Optional[Sequence[int]] = None) -> torch.Tensor:
-    """Block probabilities P [batch, hq, L/B, L/B] (fp32) of antidiagonal scoring.
+    """Block probabilities P [batch, hq, NB, NB] (fp32, NB = ceil(L/B)) of antidiagonal
+    scoring.
 
     With ``perm`` (a permutation of 0..S-1) the call is xattn_score_pattern:
     chunk i pairs query sub-row perm[i] with key sub-row i."""
     _check(Q, "Q")
     _check(K, "K", Q.dtype)
     shape = _shape_of(Q, K, B, S, causal)
-    NB = shape.L // max(shape.B, 1)
+    NB = -(-shape.L // max(shape.B, 1))
     if probs is None:
         probs = torch.empty(shape.batch, shape.hq, NB, NB, device=Q.device, dtype=torch.float32)
     _check(probs, "probs", torch.float32)
@@ -253,7 +254,7 @@ def xattn_score_select(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal:
     _check(Q, "Q")
     _check(K, "K", Q.dtype)
     shape = _shape_of(Q, K, B, S, causal)
-    NB = shape.L // max(shape.B, 1)
+    NB = -(-shape.L // max(shape.B, 1))
     want_p = probs is not None and probs is not False
     if probs is True:
         probs = torch.empty(shape.batch, shape.hq, NB, NB, device=Q.device, dtype=torch.float32)

@@ -18,7 +18,14 @@
  * - Q, K, V, O are contiguous [batch, heads, L, d] arrays. Q and O have hq
  *   heads; K and V have hkv heads. hq must be a multiple of hkv, and query
  *   head h reads KV head h / (hq / hkv) (grouped-query attention).
- * - NB = L / B query blocks and key blocks. r = B / S reshaped rows per block.
+ * - NB = ceil(L / B) query blocks and key blocks. r = B / S reshaped rows per
+ *   block. L must be a multiple of S (INVALID_ARG otherwise) but need not be a
+ *   multiple of B: the last block then holds the L - (NB-1)*B remaining tokens
+ *   (fewer reshaped rows and columns). Algorithm 1 only walks floor(L/B) whole
+ *   blocks; this extension keeps every definition below and applies it to the
+ *   tokens that exist: softmax rows run over the L/S reshaped columns, a block
+ *   probability divides by its block's own number of reshaped rows (so rows of
+ *   P still sum to 1), and attention has no query or key past L.
  * - Every call is asynchronous on the given CUDA stream (a cudaStream_t passed
  *   as void*; NULL means the legacy default stream). No call synchronises the
  *   device, except xattn_get_device_status.
@@ -65,7 +72,7 @@ typedef struct {
 
 /* Largest hq accepted (the per-head tau vector travels as a kernel argument). */
 #define XATTN_MAX_HEADS 256
-/* Largest NB = L / B accepted by xattn_select and xattn_score. */
+/* Largest NB = ceil(L / B) accepted by xattn_select and xattn_score. */
 #define XATTN_MAX_BLOCKS 4096
 
 /*
@@ -83,8 +90,9 @@ size_t xattn_score_workspace_bytes(const xattn_shape* shape);
  * and the reshaped keys are rows [K[cS], ..., K[cS+S-1]]. Let
  * x = Q_r K_r^T / sqrt(d*S). With causal != 0, reshaped column c is visible
  * to global reshaped row rho only when c <= rho. A = row softmax of x.
- * Then P[b, j] = (1/r) * (sum of A over the r x r sub-block (b, j)), so every
- * row of P sums to 1. Causal rows are 0 for j > b.
+ * Then P[b, j] = (1/r_b) * (sum of A over the sub-block (b, j)), where r_b = r
+ * for a whole block and the number of reshaped rows of a short last block, so
+ * every row of P sums to 1. Causal rows are 0 for j > b.
  *
  * Q: [batch, hq, L, d], K: [batch, hkv, L, d], both of type shape->dtype and
  *    16-byte aligned.
@@ -200,7 +208,7 @@ int xattn_sparse_attn(const void* Q, const void* K, const void* V, const xattn_s
                       const int32_t* counts, const int32_t* idx, void* O, float* lse,
                       void* ws, size_t ws_bytes, void* stream);
 
-/* Largest batch*hq*(L/B) accepted by xattn_sparse_attn_noalloc. */
+/* Largest batch*hq*NB accepted by xattn_sparse_attn_noalloc. */
 #define XATTN_NOALLOC_MAX_UNITS (1 << 18)
 
 /*
@@ -215,7 +223,7 @@ int xattn_sparse_attn(const void* Q, const void* K, const void* V, const xattn_s
  * The work order lives in a __device__ array of the library, sized for
  * XATTN_NOALLOC_MAX_UNITS work units (2 MiB). Each GPU that loads the library
  * holds it until the process exits. Returns XATTN_ERR_WORKSPACE when
- * batch*hq*(L/B) exceeds that limit.
+ * batch*hq*NB exceeds that limit.
  *
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) and caches it; make that first call before any

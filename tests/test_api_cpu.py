@@ -45,7 +45,7 @@ def test_workspace_sizes(lib):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(L=1000), -1),             # L % B != 0
+    (dict(L=1004), -1),             # L % S != 0 (L % B != 0 alone is allowed)
     (dict(S=3), -1),                # B % S != 0
     (dict(hkv=3), -1),              # hq % hkv != 0
     (dict(d=64), -2),               # bf16 needs d = 128
@@ -104,7 +104,7 @@ def test_bad_pattern_rejected(lib, perm):
 
 def test_pattern_checks_shape_and_workspace_first(lib):
     ok = (ctypes.c_int32 * 8)(*range(8))
-    bad = X.make_shape(1, 4, 2, 1000, 128, 128, 8, True, "bf16")
+    bad = X.make_shape(1, 4, 2, 1004, 128, 128, 8, True, "bf16")   # L % S != 0
     assert lib.xattn_score_pattern(FAKE, FAKE, ctypes.byref(bad), ok, FAKE, FAKE, 1 << 40,
                                    None) == -1
     s = X.make_shape(1, 4, 2, 1024, 128, 128, 8, True, "bf16")
@@ -190,3 +190,14 @@ def test_prefill_host_checks(lib):
     assert f(FAKE, FAKE, FAKE, ctypes.byref(s), good, FAKE, None, 0, odd, big, None) == -4
     wide = X.make_shape(1, 4, 2, 1024, 64, 128, 8, True, "bf16")  # bf16 needs d = 128
     assert f(FAKE, FAKE, FAKE, ctypes.byref(wide), good, FAKE, None, 0, FAKE, big, None) == -2
+
+
+def test_ragged_length_accepted(lib):
+    """L = 1000 (not a multiple of B = 128, a multiple of S = 8): 8 blocks,
+    the last of 104 tokens. The host checks pass (the call then fails only on
+    the missing workspace)."""
+    s = X.make_shape(1, 4, 2, 1000, 128, 128, 8, True, "bf16")
+    NB, r = 8, 16
+    assert X.xattn_score_workspace_bytes(s) == 4 * r * NB * (NB + 1) // 2 * 4 + 256
+    assert X.xattn_attn_workspace_bytes(s) == 8 * (4 * NB + 32)
+    assert lib.xattn_score(FAKE, FAKE, ctypes.byref(s), FAKE, None, 0, None) == -4
