@@ -7,7 +7,8 @@ attention over the selected blocks). The pages' ablation variants run
 through the same kernels: ``xattn_score_pattern`` (diagonal or random
 sampling) and ``xattn_select_topk`` / ``xattn_select_topratio`` (fixed
 budgets). ``xattn_prefill_host`` runs the whole step on host tensors with the
-host<->device copies overlapped with the compute. The library loads on first
+host<->device copies overlapped with the compute, and ``xattn_prefill_varlen``
+on a batch of sequences of different lengths. The library loads on first
 use and the calls raise if it is missing.
 """
 from .xattn import (  # noqa: F401
@@ -16,6 +17,7 @@ from .xattn import (  # noqa: F401
     library_path, EXPORTED_SYMBOLS, xattn_sparse_attn_noalloc, xattn_score_pattern,
     xattn_select_topk, xattn_select_topratio, antidiagonal_perm, diagonal_perm,
     xattn_score_select, xattn_selftest_timeout, xattn_prefill_host,
-    xattn_prefill_host_workspace_bytes,
+    xattn_prefill_host_workspace_bytes, xattn_prefill_varlen,
+    xattn_prefill_varlen_workspace_bytes,
 )
 from .pipeline import prefill_attention  # noqa: F401

@@ -23,6 +23,7 @@ __all__ = [
     "xattn_score_pattern", "xattn_select_topk", "xattn_select_topratio",
     "antidiagonal_perm", "diagonal_perm", "xattn_score_select", "xattn_selftest_timeout",
     "xattn_prefill_host_workspace_bytes", "xattn_prefill_host",
+    "xattn_prefill_varlen_workspace_bytes", "xattn_prefill_varlen",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -35,6 +36,7 @@ EXPORTED_SYMBOLS = (
     "xattn_strerror", "xattn_sparse_attn_noalloc", "xattn_score_pattern",
     "xattn_select_topk", "xattn_select_topratio", "xattn_score_select",
     "xattn_selftest_timeout", "xattn_prefill_host_workspace_bytes", "xattn_prefill_host",
+    "xattn_prefill_varlen_workspace_bytes", "xattn_prefill_varlen",
 )
 # batch * hq * (L / B) limit of xattn_sparse_attn_noalloc (XATTN_NOALLOC_MAX_UNITS)
 NOALLOC_MAX_UNITS = 1 << 18
@@ -97,6 +99,12 @@ def _lib() -> ctypes.CDLL:
         lib.xattn_prefill_host.argtypes = [vp, vp, vp, sp, ctypes.POINTER(ctypes.c_float), vp,
                                            vp, i32, vp, sz, vp]
         lib.xattn_prefill_host.restype = i32
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        lib.xattn_prefill_varlen_workspace_bytes.argtypes = [sp, i32, i32p]
+        lib.xattn_prefill_varlen_workspace_bytes.restype = sz
+        lib.xattn_prefill_varlen.argtypes = [vp, vp, vp, sp, i32, i32p,
+                                             ctypes.POINTER(ctypes.c_float), vp, vp, vp, sz, vp]
+        lib.xattn_prefill_varlen.restype = i32
         lib.xattn_selftest_timeout.argtypes = [vp]
         lib.xattn_selftest_timeout.restype = i32
         lib.xattn_get_device_status.argtypes = [vp]
@@ -415,6 +423,54 @@ def xattn_prefill_host(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, B: int
                                    int(kv_heads_per_chunk), workspace.data_ptr(),
                                    workspace.numel() * workspace.element_size(), _stream(dev))
     _raise("xattn_prefill_host", rc)
+    return (out, lse) if want_lse else out
+
+
+def xattn_prefill_varlen_workspace_bytes(shape: _Shape, seqlens: Sequence[int]) -> int:
+    arr = (ctypes.c_int32 * len(seqlens))(*[int(x) for x in seqlens])
+    return int(_lib().xattn_prefill_varlen_workspace_bytes(ctypes.byref(shape), len(seqlens),
+                                                           arr))
+
+
+def xattn_prefill_varlen(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                         seqlens: Sequence[int], hq: int, hkv: int, B: int, S: int,
+                         causal: bool, tau: Sequence[float], out: Optional[torch.Tensor] = None,
+                         lse: Optional[torch.Tensor] | bool = None,
+                         workspace: Optional[torch.Tensor] = None):
+    """The whole step on sequences of different lengths, packed one after
+    another: Q is [hq * T, d] with sequence i's [hq, L_i, d] block after the
+    previous ones (T = sum of the lengths); K and V are [hkv * T, d]. Returns O
+    packed like Q, or (O, lse) with lse [hq * T] when lse is True or a tensor."""
+    _check(Q, "Q")
+    _check(K, "K", Q.dtype)
+    _check(V, "V", Q.dtype)
+    lens = [int(x) for x in seqlens]
+    T = sum(lens)
+    if Q.dim() != 2 or Q.shape[0] != hq * T or K.shape != (hkv * T, Q.shape[1]) \
+            or V.shape != K.shape:
+        raise ValueError("expected Q [hq*T, d] and K, V [hkv*T, d] for T = sum(seqlens)")
+    shape = make_shape(1, hq, hkv, max(max(lens), 1), Q.shape[1], B, S, causal, Q.dtype)
+    if out is None:
+        out = torch.empty_like(Q)
+    _check(out, "O", Q.dtype)
+    want_lse = lse is not None and lse is not False
+    if lse is True:
+        lse = torch.empty(hq * T, device=Q.device, dtype=torch.float32)
+    if want_lse:
+        _check(lse, "lse", torch.float32)
+    taus = _per_head(tau, hq, "tau", float)
+    tarr = (ctypes.c_float * hq)(*taus)
+    larr = (ctypes.c_int32 * len(lens))(*lens)
+    need = int(_lib().xattn_prefill_varlen_workspace_bytes(ctypes.byref(shape), len(lens), larr))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
+    _check(workspace, "workspace")
+    rc = _lib().xattn_prefill_varlen(Q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                     ctypes.byref(shape), len(lens), larr, tarr, out.data_ptr(),
+                                     lse.data_ptr() if want_lse else None, workspace.data_ptr(),
+                                     workspace.numel() * workspace.element_size(),
+                                     _stream(Q.device))
+    _raise("xattn_prefill_varlen", rc)
     return (out, lse) if want_lse else out
 
 

@@ -282,6 +282,43 @@ int xattn_prefill_host(const void* Q, const void* K, const void* V, const xattn_
                        size_t ws_bytes, void* stream);
 
 /*
+ * Workspace bytes of xattn_prefill_varlen for these lengths: the scratch of
+ * the longest sequence. Returns 0 when the lengths or the shape are invalid.
+ */
+size_t xattn_prefill_varlen_workspace_bytes(const xattn_shape* shape, int nseq,
+                                            const int32_t* seqlens);
+
+/*
+ * The whole prefill step -- xattn_score_select (threshold tau), then
+ * xattn_sparse_attn -- on a batch of nseq sequences of different lengths.
+ * Sequence i has L_i = seqlens[i] tokens (HOST array; 0 skips a sequence;
+ * otherwise a multiple of S, and not necessarily of B: a short last block is
+ * handled as for a fixed-length batch). Results are bit-identical to the two
+ * calls run on sequence i alone as a batch-1 problem.
+ * Layout: the sequences are packed one after another. Sequence i of Q is a
+ * contiguous [hq, L_i, d] array starting T_i * hq * d elements into Q, with
+ * T_i = L_0 + ... + L_{i-1}; K and V hold [hkv, L_i, d] arrays at T_i * hkv *
+ * d; O is laid out like Q, and lse (optional, may be NULL) holds [hq, L_i]
+ * fp32 arrays at T_i * hq. All DEVICE pointers, 16-byte aligned for bf16.
+ * shape: hq, hkv, d, B, S, causal and dtype apply to every sequence; its
+ * batch and L are ignored.
+ * tau: HOST pointer to hq floats in (0, 1].
+ * ws / ws_bytes: DEVICE workspace of at least
+ *          xattn_prefill_varlen_workspace_bytes(shape, nseq, seqlens) bytes,
+ *          256-byte aligned; the sequences run one after another on `stream`
+ *          and share it.
+ * Errors: INVALID_ARG (NULL pointer, nseq < 1, a negative length, no
+ * non-empty sequence, a length that is not a multiple of S, bad tau),
+ * UNSUPPORTED (dtype limits, a sequence with more than XATTN_MAX_BLOCKS
+ * blocks, more than 2^31 - 1 query rows in all), WORKSPACE, CUDA. Every
+ * argument is checked before the first launch.
+ * This entry point has no counterpart in the paper.
+ */
+int xattn_prefill_varlen(const void* Q, const void* K, const void* V, const xattn_shape* shape,
+                         int nseq, const int32_t* seqlens, const float* tau, void* O,
+                         float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's status
  * word. Returns XATTN_OK, XATTN_ERR_TIMEOUT if a kernel gave up a bounded
  * wait since the last call, or XATTN_ERR_CUDA if the stream reports an error.

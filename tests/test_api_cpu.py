@@ -201,3 +201,51 @@ def test_ragged_length_accepted(lib):
     assert X.xattn_score_workspace_bytes(s) == 4 * r * NB * (NB + 1) // 2 * 4 + 256
     assert X.xattn_attn_workspace_bytes(s) == 8 * (4 * NB + 32)
     assert lib.xattn_score(FAKE, FAKE, ctypes.byref(s), FAKE, None, 0, None) == -4
+
+
+def _varlen(lib, shape, lens):
+    arr = (ctypes.c_int32 * len(lens))(*lens)
+    return lib.xattn_prefill_varlen_workspace_bytes(ctypes.byref(shape), len(lens), arr), arr
+
+
+def test_varlen_workspace_is_the_longest_sequences(lib):
+    s = X.make_shape(7, 4, 2, 1, 128, 128, 8, True, "bf16")   # batch and L are ignored
+    got, _ = _varlen(lib, s, [1000, 4096, 0, 512])
+    one = X.make_shape(1, 4, 2, 4096, 128, 128, 8, True, "bf16")
+    NB = 32
+    want = _r256(4 * NB * 1 * 4) + _r256(4 * NB * 4) + _r256(4 * NB * NB * 4) + \
+        _r256(X.xattn_score_workspace_bytes(one)) + _r256(X.xattn_attn_workspace_bytes(one))
+    assert got == want
+
+
+@pytest.mark.parametrize("lens,code", [
+    ([], -1), ([0, 0], -1), ([128, -8], -1), ([128, 100], -1),   # 100 % S != 0
+    ([128, 128 * 4097], -2),                                    # too many blocks
+])
+def test_varlen_bad_lengths(lib, lens, code):
+    s = X.make_shape(1, 4, 2, 1, 128, 128, 8, True, "bf16")
+    arr = (ctypes.c_int32 * max(len(lens), 1))(*lens)
+    assert lib.xattn_prefill_varlen_workspace_bytes(ctypes.byref(s), len(lens), arr) == 0
+    t = (ctypes.c_float * 4)(0.9, 0.9, 0.9, 0.9)
+    rc = lib.xattn_prefill_varlen(FAKE, FAKE, FAKE, ctypes.byref(s), len(lens), arr, t, FAKE,
+                                  None, FAKE, 1 << 40, None)
+    assert rc == code
+
+
+def test_varlen_host_checks(lib):
+    s = X.make_shape(1, 4, 2, 1, 128, 128, 8, True, "bf16")
+    need, arr = _varlen(lib, s, [128, 1000])
+    good = (ctypes.c_float * 4)(0.9, 0.9, 0.9, 0.9)
+    bad = (ctypes.c_float * 4)(0.9, 0.9, 1.5, 0.9)
+    f = lib.xattn_prefill_varlen
+    big = 1 << 40
+    assert f(None, FAKE, FAKE, ctypes.byref(s), 2, arr, good, FAKE, None, FAKE, big, None) == -1
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(s), 2, arr, good, None, None, FAKE, big, None) == -1
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(s), 2, arr, None, FAKE, None, FAKE, big, None) == -1
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(s), 2, arr, bad, FAKE, None, FAKE, big, None) == -1
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(s), 2, None, good, FAKE, None, FAKE, big, None) == -1
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(s), 2, arr, good, FAKE, None, None, big, None) == -4
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(s), 2, arr, good, FAKE, None, FAKE, need - 1,
+             None) == -4
+    odd = ctypes.c_void_p(0x10080)
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(s), 2, arr, good, FAKE, None, odd, big, None) == -4
