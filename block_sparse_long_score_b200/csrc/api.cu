@@ -169,11 +169,16 @@ int score_partials(const void* Q, const void* K, const Dims& D, const PermArg& p
   if (rc != XATTN_OK) return rc;
   if (D.dtype == XATTN_BF16) {
     CUtensorMap tq, tk;
+    // a CTA pair loads 128 of a tile's 256 key rows per CTA, a lone CTA all 256
+    const bool pair = D.S >= kScorePairMinS;
     if ((rc = make_map_reshaped(&tq, Q, D.S, D.R, D.batch * D.hq, 128)) != XATTN_OK) return rc;
-    if ((rc = make_map_reshaped(&tk, K, D.S, D.R, D.batch * D.hkv, 256)) != XATTN_OK) return rc;
-    if ((rc = cuda_status(launch_score_tc(D, tq, tk, perm, part, ds->status, ds->num_sms,
-                                          st))) != XATTN_OK)
+    if ((rc = make_map_reshaped(&tk, K, D.S, D.R, D.batch * D.hkv, pair ? 128 : 256)) !=
+        XATTN_OK)
       return rc;
+    const cudaError_t e =
+        pair ? launch_score_tc_pair(D, tq, tk, perm, part, ds->status, ds->num_sms, st)
+             : launch_score_tc(D, tq, tk, perm, part, ds->status, ds->num_sms, st);
+    if ((rc = cuda_status(e)) != XATTN_OK) return rc;
   } else {
     if ((rc = cuda_status(launch_score_simt(D, static_cast<const float*>(Q),
                                             static_cast<const float*>(K), perm, part, st))) !=

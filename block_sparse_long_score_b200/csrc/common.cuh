@@ -58,9 +58,19 @@ struct BudgetArg {
 // Each returns cudaSuccess or the launch error. All are asynchronous.
 
 // bf16 tensor-core scoring GEMM: partials for every (bh, rho, allowed j).
+// One CTA per 128 x 256 tile; the key map's box is 256 reshaped rows.
 cudaError_t launch_score_tc(const Dims& D, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                             const PermArg& perm, float* part, int* status, int num_sms,
                             cudaStream_t st);
+// The same partials from CTA pairs, one 256 x 256 tile per pair (M = 256
+// MMAs across two SMs); the key map's box is 128 reshaped rows.
+cudaError_t launch_score_tc_pair(const Dims& D, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                 const PermArg& perm, float* part, int* status, int num_sms,
+                                 cudaStream_t st);
+// Strides from which the pair kernel is used (a tile then has 2S >= 16
+// k-steps; with fewer, the epilogue bounds a tile and one CTA per tile is
+// faster).
+constexpr int kScorePairMinS = 8;
 
 // fp32 CUDA-core scoring, same partial layout.
 cudaError_t launch_score_simt(const Dims& D, const float* Q, const float* K,
