@@ -40,10 +40,10 @@ WORKLOAD = "c2"   # the 128K Llama-shaped layer the metric is quoted on
 # KV groups, every query block); traffic grows with the number of heads, so the
 # figures are scaled by 32 / 8 to a full call. Summaries: profiles/.
 TRAFFIC_BYTES = {
-    # score_tc 353.85 MB read + 121.10 MB written; score_reduce 134.37 + 18.82 MB
-    ("c2", "score"): 4 * (353.85 + 121.10 + 134.37 + 18.82) * 1e6,
-    # attn_tc 863.80 MB read + 238.14 MB written (sched_kernel: 1.12 MB)
-    ("c2", "sparse_attn"): 4 * (863.80 + 238.14 + 1.12) * 1e6,
+    # score_tc (CTA pairs) 382.73 MB read + 121.97 MB written; score_reduce 134.37 + 19.20 MB
+    ("c2", "score"): 4 * (382.73 + 121.97 + 134.37 + 19.20) * 1e6,
+    # attn_tc 873.24 MB read + 238.23 MB written (sched_kernel: 1.12 MB)
+    ("c2", "sparse_attn"): 4 * (873.24 + 238.23 + 1.12) * 1e6,
 }
 
 
