@@ -316,6 +316,29 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     if xattn_get_device_status(dev) != 0:
         raise RuntimeError("device status reports a kernel time-out")
 
+    # the same step captured once in a CUDA graph and replayed (what a serving
+    # loop with fixed shapes would run): launch costs paid at capture
+    graph_ms = None
+    if not args.no_graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        g.replay()
+        torch.cuda.synchronize(dev)
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        if dist:
+            torch.distributed.barrier()
+        g0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        g1.record(stream)
+        torch.cuda.synchronize(dev)
+        graph_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps, dev)
+        del g
+        if xattn_get_device_status(dev) != 0:
+            raise RuntimeError("device status reports a kernel time-out")
+
     # the same attention kernel on the full (tau = 1) mask: the dense
     # attention the block-sparse step replaces, for context
     dense_ms = None
@@ -381,6 +404,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
         "density": density,
         "per_kernel_ms": per,
         "score_select_share": (per["score"] + per["select"]) / ms_step,
+        "graph_replay_ms_per_step": graph_ms,
         "dense_mask_attn": None if dense_ms is None else {
             "ms": dense_ms,
             "tflops": dense / (dense_ms * 1e-3) / 1e12,
@@ -460,6 +484,8 @@ def main() -> None:
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="skip the CUDA-graph replay of the step reported for context")
     ap.add_argument("--no-dense", action="store_true",
                     help="skip the dense-mask attention run reported for context")
     ap.add_argument("--config", default=WORKLOAD, choices=["c1", "c2", "c3", "c4"],
