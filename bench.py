@@ -151,6 +151,73 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+class NvmlClockSampler:
+    """Samples the SM clock and the clock-event reasons through NVML every
+    ~2 ms from a host thread, so that a timed region of tens of milliseconds
+    still gets a median under load (nvidia-smi's loop starts too slowly and
+    samples too rarely for that). Reads only; changes no GPU setting."""
+
+    def __init__(self, index: int):
+        import threading
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        try:   # the CUDA device's own GPU, whatever the NVML enumeration order
+            pr = torch.cuda.get_device_properties(index)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+        self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        self.samples = []
+        self.stop_flag = threading.Event()
+        self.first = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.names = {
+            "hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+            "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+            "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+            "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap,
+        }
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, reasons))
+            except nv.NVMLError:
+                pass
+            self.first.set()
+            time.sleep(0.002)
+
+    def start(self):
+        self.thread.start()
+        self.first.wait(timeout=5)
+
+    def stop(self) -> dict:
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        sm = [m for m, _ in self.samples if m > 0]
+        reasons = sorted(n for n, bit in self.names.items()
+                         if any(r & bit for _, r in self.samples))
+        try:
+            self.nv.nvmlShutdown()
+        except self.nv.NVMLError:
+            pass
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml, 2 ms"}
+
+
+def clock_sampler(index: int):
+    """NVML polling when available, else the nvidia-smi loop."""
+    try:
+        return NvmlClockSampler(index)
+    except Exception:
+        return ClockSampler(index)
+
+
 # ------------------------------------------------------------- CPU oracle
 def oracle_sample(prob, n_blocks: int = 48) -> dict:
     """Times the fp64 oracle on one query head and an evenly spread sample of
@@ -257,7 +324,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     if dist:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    clocks = ClockSampler(local)
+    clocks = clock_sampler(local)
     clocks.start()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
