@@ -346,7 +346,7 @@ int xattn_sparse_attn(const void* Q, const void* K, const void* V, const xattn_s
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (D.dtype == XATTN_BF16) {
     unsigned long long* order = static_cast<unsigned long long*>(ws);
-    if ((rc = cuda_status(launch_sched(D, counts, idx, order, st))) != XATTN_OK) return rc;
+    if ((rc = cuda_status(launch_sched(D, counts, idx, order, ds->num_sms, st))) != XATTN_OK) return rc;
     CUtensorMap tq, tk, tv;
     if ((rc = make_map_2d(&tq, Q, static_cast<long long>(D.batch) * D.hq * D.L)) != XATTN_OK)
       return rc;

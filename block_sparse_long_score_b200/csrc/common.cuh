@@ -105,7 +105,7 @@ cudaError_t launch_select_budget(const Dims& D, const float* probs, const Budget
 // Longest-list-first order of the work units (bh, b) into `order`: one packed
 // 64-bit entry per unit (unit index, effective block count, diagonal flag).
 cudaError_t launch_sched(const Dims& D, const int32_t* counts, const int32_t* idx,
-                         unsigned long long* order, cudaStream_t st);
+                         unsigned long long* order, int num_sms, cudaStream_t st);
 
 // bf16 tensor-core block-sparse attention.
 cudaError_t launch_attn_tc(const Dims& D, const CUtensorMap& tmQ, const CUtensorMap& tmK,

@@ -77,7 +77,7 @@ extern "C" int xattn_sparse_attn_noalloc(const void* Q, const void* K, const voi
   if ((rc = device_state(&ds)) != XATTN_OK) return rc;
   unsigned long long* order = nullptr;
   if ((rc = scratch_address(&order)) != XATTN_OK) return rc;
-  if ((rc = cuda_status(launch_sched(D, counts, idx, order, st))) != XATTN_OK) return rc;
+  if ((rc = cuda_status(launch_sched(D, counts, idx, order, ds->num_sms, st))) != XATTN_OK) return rc;
   CUtensorMap tq, tk, tv;
   if ((rc = make_map_2d(&tq, Q, static_cast<long long>(D.batch) * D.hq * D.L)) != XATTN_OK)
     return rc;

@@ -68,12 +68,22 @@ __device__ __forceinline__ void unit_info8(const int32_t* __restrict__ counts,
   for (int q = 0; q < 8; ++q) n[q] = c[q];
 }
 
+// Lists at least this long on average (selected blocks per unit) make the
+// K/V reuse inside a KV-head group worth grouping the order by group; with
+// shorter lists the global longest-first order balances the CTAs better.
+constexpr int kGroupMinAvgBlocks = 48;
+
 __global__ void __launch_bounds__(kThreads)
     sched_kernel(const int32_t* __restrict__ counts, const int32_t* __restrict__ idx, int units,
-                 int NB, int causal, int ragged, unsigned long long* __restrict__ order) {
-  extern __shared__ int hist[];  // NB + 1 bins, bin = NB - count
-  const int nbins = NB + 1;
-  for (int i = threadIdx.x; i < nbins; i += kThreads) hist[i] = 0;
+                 int NB, int causal, int ragged, int groups, int units_per_group, int ctas,
+                 unsigned long long* __restrict__ order) {
+  // plain[NB - count] counts units by length; grouped[g * (NB + 1) + NB - count]
+  // by KV-head group and length (only when there is more than one group)
+  extern __shared__ int bins[];
+  int* plain = bins;
+  int* grouped = bins + (NB + 1);
+  const int ngrouped = groups > 1 ? groups * (NB + 1) : 0;
+  for (int i = threadIdx.x; i < NB + 1 + ngrouped; i += kThreads) bins[i] = 0;
   __syncthreads();
   // 8 units per thread per batch: their load chains overlap
   for (int u0 = 0; u0 < units; u0 += 8 * kThreads) {
@@ -81,18 +91,37 @@ __global__ void __launch_bounds__(kThreads)
     bool diag[8];
     unit_info8(counts, idx, u0 + threadIdx.x, units, NB, causal, ragged, n, diag);
 #pragma unroll
-    for (int q = 0; q < 8; ++q)
-      if (u0 + threadIdx.x + q * kThreads < units) atomicAdd(&hist[NB - n[q]], 1);
+    for (int q = 0; q < 8; ++q) {
+      const int u = u0 + threadIdx.x + q * kThreads;
+      if (u >= units) continue;
+      atomicAdd(&plain[NB - n[q]], 1);
+      if (ngrouped) atomicAdd(&grouped[(u / units_per_group) * (NB + 1) + NB - n[q]], 1);
+    }
   }
   __syncthreads();
-  // exclusive scan of the bins: each thread sums a contiguous chunk
+  // total selected blocks, from the length histogram
+  __shared__ long long blk_tot[kThreads / 32];
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  long long blocks = 0;
+  for (int i = threadIdx.x; i < NB + 1; i += kThreads)
+    blocks += static_cast<long long>(plain[i]) * (NB - i);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) blocks += __shfl_xor_sync(0xffffffffu, blocks, o);
+  if (lane == 0) blk_tot[warp] = blocks;
+  __syncthreads();
+  long long total = 0;
+  for (int w = 0; w < kThreads / 32; ++w) total += blk_tot[w];
+  const bool by_group =
+      ngrouped > 0 && total >= static_cast<long long>(kGroupMinAvgBlocks) * units;
+  int* hist = by_group ? grouped : plain;
+  const int nbins = by_group ? ngrouped : NB + 1;
+  // exclusive scan of the chosen bins: each thread sums a contiguous chunk
   __shared__ int warp_tot[kThreads / 32];
   const int per = (nbins + kThreads - 1) / kThreads;
   const int lo = threadIdx.x * per;
   const int hi = min(lo + per, nbins);
   int local = 0;
   for (int i = lo; i < hi; ++i) local += hist[i];
-  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
   int incl = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -127,7 +156,17 @@ __global__ void __launch_bounds__(kThreads)
     for (int q = 0; q < 8; ++q) {
       const int u = u0 + threadIdx.x + q * kThreads;
       if (u >= units) continue;
-      const int pos = atomicAdd(&hist[NB - n[q]], 1);
+      const int bin = by_group ? (u / units_per_group) * (NB + 1) + NB - n[q] : NB - n[q];
+      int pos = atomicAdd(&hist[bin], 1);
+      // the attention CTAs deal the order out in rounds of `ctas` units (CTA
+      // i takes entries i, i + ctas, ...); every other round runs backwards,
+      // so the CTA that gets a round's longest unit gets the next round's
+      // shortest
+      const int round = pos / ctas;
+      if (round & 1) {
+        const int m = min(ctas, units - round * ctas);
+        pos = round * ctas + (m - 1 - (pos - round * ctas));
+      }
       order[pos] = static_cast<unsigned long long>(static_cast<uint32_t>(u)) |
                    (static_cast<unsigned long long>(n[q]) << 32) |
                    (static_cast<unsigned long long>(diag[q] ? 1 : 0) << 48);
@@ -138,11 +177,27 @@ __global__ void __launch_bounds__(kThreads)
 }  // namespace
 
 cudaError_t launch_sched(const Dims& D, const int32_t* counts, const int32_t* idx,
-                         unsigned long long* order, cudaStream_t st) {
+                         unsigned long long* order, int num_sms, cudaStream_t st) {
   const int units = D.batch * D.hq * D.NB;
-  const size_t smem = static_cast<size_t>(D.NB + 1) * sizeof(int);
+  // With long lists, units are grouped by KV head (the hq/hkv query heads
+  // that share one K/V), longest list first inside a group: the persistent
+  // CTAs take units round-robin, so they all work on one group's K/V at a
+  // time, which stays in L2, instead of every KV head at once. The kernel
+  // makes the choice from the counts (kGroupMinAvgBlocks).
+  int groups = D.batch * D.hkv;
+  const int per_group = D.group * D.NB;  // units of one KV head (unit = bh * NB + qb)
+  if (static_cast<size_t>(groups + 1) * (D.NB + 1) * sizeof(int) > 160 * 1024)
+    groups = 1;  // too many bins for shared memory: the plain order only
+  const size_t smem =
+      static_cast<size_t>(groups > 1 ? groups + 1 : 1) * (D.NB + 1) * sizeof(int);
+  cudaError_t e = cudaFuncSetAttribute(sched_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  // the attention kernel runs min(SMs, units) persistent CTAs
+  const int ctas = num_sms < units ? num_sms : (units > 0 ? units : 1);
   sched_kernel<<<1, kThreads, smem, st>>>(counts, idx, units, D.NB, D.causal,
-                                          D.tail != D.B ? 1 : 0, order);
+                                          D.tail != D.B ? 1 : 0, groups, per_group, ctas,
+                                          order);
   return cudaGetLastError();
 }
 
