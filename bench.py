@@ -40,10 +40,10 @@ WORKLOAD = "c2"   # the 128K Llama-shaped layer the metric is quoted on
 # KV groups, every query block); traffic grows with the number of heads, so the
 # figures are scaled by 32 / 8 to a full call. Summaries: profiles/.
 TRAFFIC_BYTES = {
-    # score_tc (CTA pairs) 382.73 MB read + 121.97 MB written; score_reduce 134.37 + 19.20 MB
-    ("c2", "score"): 4 * (382.73 + 121.97 + 134.37 + 19.20) * 1e6,
-    # attn_tc 873.24 MB read + 238.23 MB written (sched_kernel: 1.12 MB)
-    ("c2", "sparse_attn"): 4 * (873.24 + 238.23 + 1.12) * 1e6,
+    # score_tc (CTA pairs) 390.05 MB read + 122.84 MB written; score_reduce 134.37 + 18.59 MB
+    ("c2", "score"): 4 * (390.05 + 122.84 + 134.37 + 18.59) * 1e6,
+    # attn_tc 864.53 MB read + 237.99 MB written (sched_kernel: 1.14 MB)
+    ("c2", "sparse_attn"): 4 * (864.53 + 237.99 + 1.14) * 1e6,
 }
 
 
