@@ -202,7 +202,11 @@ size_t xattn_attn_workspace_bytes(const xattn_shape* shape);
  * lse: out, optional (may be NULL), fp32 [batch, hq, L], natural-log
  *      log-sum-exp of each row's scaled logits.
  * ws / ws_bytes: at least xattn_attn_workspace_bytes(shape).
- * The work units (batch, h, b) run longest-list-first on persistent CTAs.
+ * The work units (batch, h, b) run on persistent CTAs, longest list first,
+ * dealt in serpentine rounds; when the lists average at least 48 blocks the
+ * order is grouped by KV head first (one head's K/V at a time stays in L2).
+ * The order changes only the speed: every unit's output is the same.
+ * Every call is capturable in a CUDA graph.
  */
 int xattn_sparse_attn(const void* Q, const void* K, const void* V, const xattn_shape* shape,
                       const int32_t* counts, const int32_t* idx, void* O, float* lse,
