@@ -1,10 +1,14 @@
-// sched.cu -- longest-list-first order of the sparse-attention work units.
+// sched.cu -- the order in which the persistent attention CTAs take the
+// sparse-attention work units.
 //
 // A work unit is one (batch*head, query block) pair; its cost is proportional
 // to its number of selected key blocks. Causal lists grow with the query-block
 // index, so the units are ordered by block count, descending (a counting sort
-// over counts 0..NB in one CTA). The persistent attention CTAs take units
-// round-robin from this order, which spreads the long lists first.
+// over counts 0..NB in one CTA). The CTAs take entries round-robin, and every
+// other round of the order is reversed (serpentine), so the long lists are
+// spread first and evenly. When the lists are long on average, the order is
+// grouped by KV head first, so that all CTAs work on one head's K/V at a
+// time (it stays in L2); the kernel decides from the count histogram.
 //
 // Each order entry packs everything the attention kernel needs to start a
 // unit into one 64-bit word, so that it costs one (prefetchable) load:

@@ -13,6 +13,10 @@
 // the diagonal (s = i) and random-permutation patterns of the sparsity-pattern
 // ablation (Knowl 9 of the chapterpal page, §3.4 Ablation Study).
 //
+// This kernel serves the short strides (S < 8: at most 8 k-steps of 64
+// features a tile, where the epilogue, not the tensor core, bounds a tile);
+// score_tc_pair.cu runs the longer ones on CTA pairs.
+//
 // Tiles are 128 (rho) x 256 (c), accumulated in TMEM (fp32), two accumulators
 // (512 columns) so the epilogue of one tile overlaps the MMAs of the next.
 // The epilogue never stores x: for each row it reduces every key block's r
