@@ -287,7 +287,9 @@ int xattn_prefill_host(const void* Q, const void* K, const void* V, const xattn_
 
 /*
  * Workspace bytes of xattn_prefill_varlen for these lengths: the scratch of
- * the longest sequence. Returns 0 when the lengths or the shape are invalid.
+ * the longest sequence, once for each concurrent lane (one lane per non-empty
+ * sequence, at most four). Returns 0 when the lengths or the shape are
+ * invalid.
  */
 size_t xattn_prefill_varlen_workspace_bytes(const xattn_shape* shape, int nseq,
                                             const int32_t* seqlens);
@@ -309,8 +311,12 @@ size_t xattn_prefill_varlen_workspace_bytes(const xattn_shape* shape, int nseq,
  * tau: HOST pointer to hq floats in (0, 1].
  * ws / ws_bytes: DEVICE workspace of at least
  *          xattn_prefill_varlen_workspace_bytes(shape, nseq, seqlens) bytes,
- *          256-byte aligned; the sequences run one after another on `stream`
- *          and share it.
+ *          256-byte aligned.
+ * The sequences are dealt round-robin over up to four lanes that run
+ * concurrently (a short sequence's kernels leave most SMs free): lane 0 is
+ * `stream`, the others are streams the call creates, forked off `stream` with
+ * an event and joined back into it, so the call is ordered on `stream` like
+ * any other. Each lane has its own part of the workspace.
  * Errors: INVALID_ARG (NULL pointer, nseq < 1, a negative length, no
  * non-empty sequence, a length that is not a multiple of S, bad tau),
  * UNSUPPORTED (dtype limits, a sequence with more than XATTN_MAX_BLOCKS

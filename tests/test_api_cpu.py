@@ -208,14 +208,16 @@ def _varlen(lib, shape, lens):
     return lib.xattn_prefill_varlen_workspace_bytes(ctypes.byref(shape), len(lens), arr), arr
 
 
-def test_varlen_workspace_is_the_longest_sequences(lib):
+def test_varlen_workspace_is_the_longest_sequences_per_lane(lib):
     s = X.make_shape(7, 4, 2, 1, 128, 128, 8, True, "bf16")   # batch and L are ignored
     got, _ = _varlen(lib, s, [1000, 4096, 0, 512])
     one = X.make_shape(1, 4, 2, 4096, 128, 128, 8, True, "bf16")
     NB = 32
-    want = _r256(4 * NB * 1 * 4) + _r256(4 * NB * 4) + _r256(4 * NB * NB * 4) + \
+    lane = _r256(4 * NB * 1 * 4) + _r256(4 * NB * 4) + _r256(4 * NB * NB * 4) + \
         _r256(X.xattn_score_workspace_bytes(one)) + _r256(X.xattn_attn_workspace_bytes(one))
-    assert got == want
+    assert got == 3 * lane                       # three non-empty sequences: three lanes
+    many, _ = _varlen(lib, s, [4096] + [128] * 9)
+    assert many == 4 * lane                      # at most four lanes
 
 
 @pytest.mark.parametrize("lens,code", [

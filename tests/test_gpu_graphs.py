@@ -91,7 +91,8 @@ def test_fused_call_and_varlen_replay_in_a_graph():
     eager = out.clone()
     out.zero_()
     g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
+    # the call forks its lanes' streams while the capture runs
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
         xattn_prefill_varlen(Q, K, V, lens, 2, 1, 128, 8, True, tau, out=out)
     g.replay()
     torch.cuda.synchronize()
