@@ -38,7 +38,7 @@ EXPORTED_SYMBOLS = (
     "xattn_selftest_timeout", "xattn_prefill_host_workspace_bytes", "xattn_prefill_host",
     "xattn_prefill_varlen_workspace_bytes", "xattn_prefill_varlen",
 )
-# batch * hq * (L / B) limit of xattn_sparse_attn_noalloc (XATTN_NOALLOC_MAX_UNITS)
+# batch * hq * NB limit of xattn_sparse_attn_noalloc (XATTN_NOALLOC_MAX_UNITS)
 NOALLOC_MAX_UNITS = 1 << 18
 
 
