@@ -12,12 +12,10 @@ import numpy as np
 import pytest
 import torch
 
-import oracle.xattn_oracle as O
 from block_sparse_long_score_b200 import (xattn_get_device_status, xattn_prefill_host,
                                           xattn_score, xattn_score_select, xattn_select,
                                           xattn_sparse_attn, xattn_sparse_attn_noalloc)
 from block_sparse_long_score_b200.synth import make_problem
-from tests import parity as PT
 from tests.test_gpu_parity import check_problem, run_gpu, sample_blocks
 
 pytestmark = pytest.mark.gpu

@@ -3,7 +3,6 @@ the max-over-ranks timing reduction. The path itself has no collective."""
 import os
 import socket
 
-import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp

@@ -7,7 +7,6 @@ with the ordinary entry point's, which takes a caller-allocated workspace.
 This file is collected last on purpose, so a stop-at-first-failure run has
 already run every other test.
 """
-import numpy as np
 import pytest
 import torch
 
