@@ -23,7 +23,7 @@ __all__ = [
     "xattn_score_pattern", "xattn_select_topk", "xattn_select_topratio",
     "antidiagonal_perm", "diagonal_perm", "xattn_score_select", "xattn_selftest_timeout",
     "xattn_prefill_host_workspace_bytes", "xattn_prefill_host",
-    "xattn_prefill_varlen_workspace_bytes", "xattn_prefill_varlen",
+    "xattn_prefill_varlen_workspace_bytes", "xattn_prefill_varlen", "xattn_check_lists",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -36,7 +36,7 @@ EXPORTED_SYMBOLS = (
     "xattn_strerror", "xattn_sparse_attn_noalloc", "xattn_score_pattern",
     "xattn_select_topk", "xattn_select_topratio", "xattn_score_select",
     "xattn_selftest_timeout", "xattn_prefill_host_workspace_bytes", "xattn_prefill_host",
-    "xattn_prefill_varlen_workspace_bytes", "xattn_prefill_varlen",
+    "xattn_prefill_varlen_workspace_bytes", "xattn_prefill_varlen", "xattn_check_lists",
 )
 # batch * hq * NB limit of xattn_sparse_attn_noalloc (XATTN_NOALLOC_MAX_UNITS)
 NOALLOC_MAX_UNITS = 1 << 18
@@ -105,6 +105,8 @@ def _lib() -> ctypes.CDLL:
         lib.xattn_prefill_varlen.argtypes = [vp, vp, vp, sp, i32, i32p,
                                              ctypes.POINTER(ctypes.c_float), vp, vp, vp, sz, vp]
         lib.xattn_prefill_varlen.restype = i32
+        lib.xattn_check_lists.argtypes = [vp, vp, sp, vp, vp]
+        lib.xattn_check_lists.restype = i32
         lib.xattn_selftest_timeout.argtypes = [vp]
         lib.xattn_selftest_timeout.restype = i32
         lib.xattn_get_device_status.argtypes = [vp]
@@ -372,6 +374,29 @@ def xattn_sparse_attn_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                                           _stream(Q.device))
     _raise("xattn_sparse_attn_noalloc", rc)
     return out
+
+
+def xattn_check_lists(Q: torch.Tensor, K: torch.Tensor, counts: torch.Tensor, idx: torch.Tensor,
+                      B: int, causal: bool, bad: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Counts the rows of (counts, idx) that break the list layout
+    xattn_sparse_attn expects (counts in [0, NB], entries strictly ascending
+    in [0, NB)). Q and K give the shape only. Returns a one-element int32
+    device tensor (``bad`` if given), written on the current stream."""
+    _check(Q, "Q")
+    _check(K, "K", Q.dtype)
+    _check(counts, "counts", torch.int32)
+    _check(idx, "idx", torch.int32)
+    shape = _shape_of(Q, K, B, 1, causal)
+    rows = shape.batch * shape.hq * -(-shape.L // shape.B)
+    if counts.numel() != rows or idx.numel() != rows * -(-shape.L // shape.B):
+        raise ValueError("counts / idx do not match the shape")
+    if bad is None:
+        bad = torch.empty(1, device=Q.device, dtype=torch.int32)
+    _check(bad, "bad", torch.int32)
+    rc = _lib().xattn_check_lists(counts.data_ptr(), idx.data_ptr(), ctypes.byref(shape),
+                                  bad.data_ptr(), _stream(Q.device))
+    _raise("xattn_check_lists", rc)
+    return bad
 
 
 def xattn_prefill_host_workspace_bytes(shape: _Shape, kv_heads_per_chunk: int = 0) -> int:

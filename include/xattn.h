@@ -241,6 +241,26 @@ int xattn_sparse_attn_noalloc(const void* Q, const void* K, const void* V,
                               const int32_t* idx, void* O, float* lse, void* stream);
 
 /*
+ * Validates block lists made outside xattn_select before they go to
+ * xattn_sparse_attn. That call trusts the layout xattn_select writes: each
+ * counts[batch, h, b] is in [0, NB], and the first counts[batch, h, b]
+ * entries of idx[batch, h, b, :] are strictly ascending block indices in
+ * [0, NB) (causal rows may end in blocks above the diagonal; the attention
+ * drops those). A list that breaks it gives wrong rows but no out-of-bounds
+ * access. This entry point has no counterpart in the paper.
+ *
+ * counts, idx: device, [batch, hq, NB] and [batch, hq, NB, NB] int32 (entries
+ *              past a row's count are not read).
+ * bad_rows: device, one int32; the call sets it to the number of rows that
+ *           break the layout (0 for valid lists). Read it after the stream
+ *           has reached it. Owned by the caller.
+ * Returns XATTN_ERR_INVALID_ARG for a bad shape or a NULL pointer, else the
+ * launch status. Capturable in a CUDA graph.
+ */
+int xattn_check_lists(const int32_t* counts, const int32_t* idx, const xattn_shape* shape,
+                      int32_t* bad_rows, void* stream);
+
+/*
  * Workspace bytes of xattn_prefill_host for a shape and a chunk size (see
  * below). Returns 0 for an invalid shape or chunk size.
  */

@@ -251,3 +251,14 @@ def test_varlen_host_checks(lib):
              None) == -4
     odd = ctypes.c_void_p(0x10080)
     assert f(FAKE, FAKE, FAKE, ctypes.byref(s), 2, arr, good, FAKE, None, odd, big, None) == -4
+
+
+def test_check_lists_host_checks(lib):
+    """xattn_check_lists rejects a bad shape or a NULL pointer before any CUDA call."""
+    s = X.make_shape(1, 2, 2, 1024, 128, 128, 1, True, "bf16")
+    bad = X.make_shape(1, 2, 2, 1004, 128, 128, 8, True, "bf16")   # L not a multiple of S
+    assert lib.xattn_check_lists(FAKE, FAKE, ctypes.byref(bad), FAKE, None) == -1
+    assert lib.xattn_check_lists(None, FAKE, ctypes.byref(s), FAKE, None) == -1
+    assert lib.xattn_check_lists(FAKE, None, ctypes.byref(s), FAKE, None) == -1
+    assert lib.xattn_check_lists(FAKE, FAKE, ctypes.byref(s), None, None) == -1
+    assert lib.xattn_check_lists(FAKE, FAKE, None, FAKE, None) == -1
