@@ -504,7 +504,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
         # the same copies and calls one after another on one stream, for context
         "e2e_serial": {"value": whole_job_ms_per_layer(e2e_serial_ms, world),
                        "unit": "ms/layer"},
-        "gpu_launches": (4 if args.fused else 5) * args.steps,
+        "gpu_launches": (4 if args.fused else 6) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -269,7 +269,7 @@ int xattn_select(const float* probs, const float* tau, const xattn_shape* shape,
   DeviceState* ds = nullptr;
   if ((rc = device_state(&ds)) != XATTN_OK) return rc;
   return cuda_status(
-      launch_select(D, probs, ta, mask, counts, idx, static_cast<cudaStream_t>(stream)));
+      launch_select(D, probs, ta, mask, counts, idx, ds->num_sms, static_cast<cudaStream_t>(stream)));
 }
 
 int xattn_score_select(const void* Q, const void* K, const xattn_shape* shape, const float* tau,

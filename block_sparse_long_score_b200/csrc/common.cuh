@@ -84,9 +84,10 @@ struct TauArg {
   float v[XATTN_MAX_HEADS];
 };
 
-// find_blocks on every row of P.
+// find_blocks on every row of P (a register-only walk of the ranking, then
+// the histogram search on the rows it leaves; num_sms sizes that second grid).
 cudaError_t launch_select(const Dims& D, const float* probs, const TauArg& tau, uint32_t* mask,
-                          int32_t* counts, int32_t* idx, cudaStream_t st);
+                          int32_t* counts, int32_t* idx, int num_sms, cudaStream_t st);
 
 // partials -> P (optional) and find_blocks, fused (same outputs as
 // launch_score_reduce followed by launch_select).

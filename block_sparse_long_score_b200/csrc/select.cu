@@ -149,19 +149,161 @@ __global__ void __launch_bounds__(kBudgetWarps * 32)
   emit_row(keys, n, NB, take_all, vstar, icut, row, lane, mask, counts, idx);
 }
 
-__global__ void __launch_bounds__(kThreads)
-    select_kernel(const float* __restrict__ probs, const TauArg tau, int NB, int hq, int causal,
-                  long long rows, int nb_stage, uint32_t* __restrict__ mask,
-                  int32_t* __restrict__ counts, int32_t* __restrict__ idx) {
-  extern __shared__ __align__(16) uint8_t smem[];
+// ---------------------------------------------------------------------------
+// find_blocks in two kernels.
+//
+// select_fast_kernel (one warp per row, no shared memory, so up to 64 rows in
+// flight per SM): while reading the row each lane keeps its kTop best blocks in
+// the find_blocks ranking (probability descending, index ascending) as 64-bit
+// rank keys in registers. Every block missing from those lists ranks at or
+// below `bound`, the best of the lanes' kTop-th entries. So taking the best
+// list head across the warp, again and again, walks the row's ranking exactly
+// for every block ranked above `bound`, and adds the probabilities in that
+// order in fp64: the same sequential sum the definition takes. If the sum
+// reaches tau above `bound`, that block is the cut. If every lane holds fewer
+// than kTop blocks, the walk covers the whole row, and a row whose sum never
+// reaches tau takes every block. Otherwise the row is marked (count -1) for
+// select_fallback_kernel, the histogram search of select_core.cuh, which runs
+// on the marked rows only. Rows with a few dominant blocks -- the long-context
+// case -- almost all finish in the fast kernel; rows whose lanes' two best
+// blocks sum to less than tau need many blocks and skip the walk.
+constexpr int kFastWarps = 8;
+constexpr int kTop = 5;
+
+// Rank key of block j with fp32 bits k (sign cleared): larger ranks first.
+// ~j keeps the lower index first among equal values, and no block has key 0.
+__device__ __forceinline__ unsigned long long rank_key(uint32_t k, int j) {
+  return (static_cast<unsigned long long>(k) << 32) | static_cast<uint32_t>(~j);
+}
+
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long y = __shfl_xor_sync(0xffffffffu, v, o);
+    v = y > v ? y : v;
+  }
+  return v;
+}
+
+__global__ void __launch_bounds__(kFastWarps * 32)
+    select_fast_kernel(const float* __restrict__ probs, const TauArg tau, int NB, int hq,
+                       int causal, long long rows, uint32_t* __restrict__ mask,
+                       int32_t* __restrict__ counts, int32_t* __restrict__ idx) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const long long row = static_cast<long long>(blockIdx.x) * kWarps + warp;
+  const long long row = static_cast<long long>(blockIdx.x) * kFastWarps + warp;
   if (row >= rows) return;
 
-  uint8_t* wbase = smem + static_cast<size_t>(warp) * (sizeof(WarpSmem) + nb_stage * 4);
-  WarpSmem& W = *reinterpret_cast<WarpSmem*>(wbase);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(wbase + sizeof(WarpSmem));
+  const long long bh = row / NB;
+  const int b = static_cast<int>(row % NB);
+  const int h = static_cast<int>(bh % hq);
+  const int n = causal ? b + 1 : NB;
+  const double t = static_cast<double>(tau.v[h]);
+  const float* prow = probs + row * NB;
 
+  bool take_all = t >= 1.0;
+  unsigned long long cut = 0;  // rank key of the cut block: blocks ranked >= cut are chosen
+  if (!take_all) {
+    unsigned long long c[kTop];
+#pragma unroll
+    for (int i = 0; i < kTop; ++i) c[i] = 0ull;
+    for (int j0 = 0; j0 < n; j0 += 8 * 32) {
+      uint32_t v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * 32 + lane;
+        v[u] = j < n ? __float_as_uint(__ldg(prow + j)) & 0x7FFFFFFFu : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * 32 + lane;
+        if (j < n) {
+          unsigned long long x = rank_key(v[u], j);
+#pragma unroll
+          for (int i = 0; i < kTop; ++i) {  // insertion into the descending list
+            const unsigned long long y = c[i];
+            c[i] = x > y ? x : y;
+            x = x > y ? y : x;
+          }
+        }
+      }
+    }
+    const unsigned long long bound = warp_max_u64(c[kTop - 1]);
+    // The lanes' two best entries are 64 distinct blocks, so the row's 64 best
+    // blocks hold at least their mass: if that reaches tau, the cut is among
+    // the first 64 of the walk. Otherwise the row needs many blocks (a flat
+    // row), and it goes straight to the histogram search instead of walking.
+    const double heads =
+        warp_sum_d(static_cast<double>(__uint_as_float(static_cast<uint32_t>(c[0] >> 32))) +
+                   static_cast<double>(__uint_as_float(static_cast<uint32_t>(c[1] >> 32))));
+    double acc = 0.0;
+    bool decided = false;
+    // at most kTop - 1 blocks a lane rank above bound
+    for (int it = 0; it < 32 * kTop && (heads >= t || bound == 0ull); ++it) {
+      const unsigned long long m = warp_max_u64(c[0]);
+      if (m <= bound) break;  // includes m == 0: the lists are empty
+      acc += static_cast<double>(__uint_as_float(static_cast<uint32_t>(m >> 32)));
+      if (c[0] == m) {  // the owner lane pops its head
+#pragma unroll
+        for (int i = 0; i + 1 < kTop; ++i) c[i] = c[i + 1];
+        c[kTop - 1] = 0ull;
+      }
+      if (acc >= t) {
+        cut = m;
+        decided = true;
+        break;
+      }
+    }
+    if (!decided) {
+      if (bound != 0ull) {  // the cut lies at or below bound: the histogram search decides
+        if (lane == 0) counts[row] = -1;
+        return;
+      }
+      take_all = true;  // the whole row was walked and its sum stays below tau
+    }
+  }
+
+  // emit: mask words over all NB columns, the index list in ascending order
+  const int Wn = (NB + 31) / 32;
+  uint32_t* mrow = mask + row * Wn;
+  int32_t* irow = idx + row * NB;
+  const unsigned lt = (1u << lane) - 1u;
+  int running = 0;
+  for (int j0 = 0; j0 < Wn * 32; j0 += 8 * 32) {
+    bool sel[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * 32 + lane;
+      sel[u] = false;
+      if (j < n) {
+        if (take_all) {
+          sel[u] = true;
+        } else {
+          const uint32_t k = __float_as_uint(__ldg(prow + j)) & 0x7FFFFFFFu;
+          sel[u] = rank_key(k, j) >= cut;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int w = j0 / 32 + u;
+      if (w >= Wn) break;
+      const unsigned sb = __ballot_sync(0xffffffffu, sel[u]);
+      if (lane == 0) mrow[w] = sb;
+      if (sel[u]) irow[running + __popc(sb & lt)] = w * 32 + lane;
+      running += __popc(sb);
+    }
+  }
+  if (lane == 0) counts[row] = running;
+}
+
+// The histogram search of one row (select_core.cuh), with its keys staged in
+// the warp's shared memory.
+__device__ __forceinline__ void select_row_hist(const float* __restrict__ probs, const TauArg& tau,
+                                                int NB, int hq, int causal, long long row,
+                                                WarpSmem& W, uint32_t* keys, int lane,
+                                                uint32_t* __restrict__ mask,
+                                                int32_t* __restrict__ counts,
+                                                int32_t* __restrict__ idx) {
   const long long bh = row / NB;
   const int b = static_cast<int>(row % NB);
   const int h = static_cast<int>(bh % hq);
@@ -198,6 +340,32 @@ __global__ void __launch_bounds__(kThreads)
   int icut;
   sel::find_cut(keys, n, t, tot, kmax, W, lane, take_all, vstar, icut);
   emit_row(keys, n, NB, take_all, vstar, icut, row, lane, mask, counts, idx);
+  __syncwarp();  // the keys are overwritten by the warp's next row
+}
+
+// Persistent: warp g of G owns rows g, g + G, g + 2G, ... and runs the
+// histogram search on those the fast kernel marked.
+__global__ void __launch_bounds__(kThreads)
+    select_fallback_kernel(const float* __restrict__ probs, const TauArg tau, int NB, int hq,
+                           int causal, long long rows, int nb_stage, uint32_t* __restrict__ mask,
+                           int32_t* __restrict__ counts, int32_t* __restrict__ idx) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  uint8_t* wbase = smem + static_cast<size_t>(warp) * (sizeof(WarpSmem) + nb_stage * 4);
+  WarpSmem& W = *reinterpret_cast<WarpSmem*>(wbase);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(wbase + sizeof(WarpSmem));
+
+  const long long G = static_cast<long long>(gridDim.x) * kWarps;
+  const long long g = static_cast<long long>(blockIdx.x) * kWarps + warp;
+  for (long long r0 = g; r0 < rows; r0 += 32 * G) {
+    const long long r = r0 + lane * G;
+    unsigned todo = __ballot_sync(0xffffffffu, r < rows && counts[r] < 0);
+    while (todo) {
+      const int q = __ffs(todo) - 1;
+      todo &= todo - 1;
+      select_row_hist(probs, tau, NB, hq, causal, r0 + q * G, W, keys, lane, mask, counts, idx);
+    }
+  }
 }
 
 }  // namespace
@@ -219,15 +387,27 @@ cudaError_t launch_select_budget(const Dims& D, const float* probs, const Budget
 }
 
 cudaError_t launch_select(const Dims& D, const float* probs, const TauArg& tau, uint32_t* mask,
-                          int32_t* counts, int32_t* idx, cudaStream_t st) {
+                          int32_t* counts, int32_t* idx, int num_sms, cudaStream_t st) {
   const long long rows = static_cast<long long>(D.batch) * D.hq * D.NB;
+  const long long fast_grid = (rows + kFastWarps - 1) / kFastWarps;
+  select_fast_kernel<<<static_cast<unsigned>(fast_grid), kFastWarps * 32, 0, st>>>(
+      probs, tau, D.NB, D.hq, D.causal, rows, mask, counts, idx);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
   const int nb_stage = (D.NB + 3) & ~3;
   const size_t smem = static_cast<size_t>(kWarps) * (sizeof(WarpSmem) + nb_stage * 4);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  e = cudaFuncSetAttribute(select_fallback_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const long long grid = (rows + kWarps - 1) / kWarps;
-  select_kernel<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_fallback_kernel, kThreads,
+                                                    smem);
+  if (e != cudaSuccess) return e;
+  const long long full = static_cast<long long>(num_sms) * (per_sm > 0 ? per_sm : 1);
+  const long long need = (rows + kWarps - 1) / kWarps;
+  const long long grid = need < full ? need : full;
+  select_fallback_kernel<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(
       probs, tau, D.NB, D.hq, D.causal, rows, nb_stage, mask, counts, idx);
   return cudaGetLastError();
 }
