@@ -3,12 +3,15 @@
 // smallest set of blocks whose probability mass reaches tau), and the
 // fixed-budget Top-K / Top-Ratio selection of the pages' ablation.
 //
-// One warp per row. The row's fp32 bit patterns (monotone in value for
-// p >= 0) are staged in shared memory and summed in fp64; the cut search
-// (octave histograms refined on the mantissa bits) is in select_core.cuh,
-// shared with the fused score->select kernel. All sums are fp64, so the choice
-// matches a sequential fp64 walk of the ranked row up to rounding in the last
-// bits.
+// find_blocks runs as two kernels, one warp per row in each. The first walks
+// the row's ranking from per-lane top lists held in registers and adds the
+// probabilities in fp64 in ranked order, exactly as the definition does; it
+// decides almost every row of a long-context layer. The rows it cannot decide
+// go to the second, which stages the row's fp32 bit patterns (monotone in
+// value for p >= 0) in shared memory and runs the histogram search of
+// select_core.cuh (shared with the fused score->select kernel). Its sums are
+// fp64 too, so its choice matches the sequential fp64 walk up to rounding in
+// the last bits.
 #include "select_core.cuh"
 
 namespace xattn {
