@@ -1,10 +1,13 @@
 """xattn_score_select (scoring, block sums and find_blocks in one call)
 against xattn_score followed by xattn_select.
 
-The fused kernel computes each row of P with the reduce kernel's arithmetic
-and runs the selection kernel's cut search on it, so on the same inputs both
-paths must agree bit for bit: P (when requested), masks, counts and lists.
-The two-call path is itself checked against the oracle in the parity tests.
+The fused kernel computes each row of P with the reduce kernel's arithmetic,
+so P is bit-identical. Its cut comes from the histogram search, while the
+two-call path first walks the ranking in order; both add the probabilities
+in fp64, so they can differ only where a running sum lies within a rounding
+step of tau, which no row of these inputs does. Masks, counts and lists must
+therefore agree bit for bit. The two-call path is itself checked against the
+oracle in the parity tests.
 """
 import numpy as np
 import pytest
