@@ -40,6 +40,15 @@
  * antidiagonal) and xattn_select_topk / xattn_select_topratio (fixed budgets
  * instead of the threshold).
  *
+ * The remaining calls have no counterpart in the paper; each is documented
+ * where it is declared:
+ *   xattn_score_select         scoring and find_blocks in one call (P kept on chip)
+ *   xattn_sparse_attn_noalloc  the attention without a workspace
+ *   xattn_check_lists          validation of block lists made by the caller
+ *   xattn_prefill_host         the whole step on HOST buffers (the one call
+ *                              whose tensors may live in host memory)
+ *   xattn_prefill_varlen       the whole step on packed variable-length sequences
+ *
  * Data types: XATTN_BF16 runs the tensor-core (tcgen05) kernels and needs
  * d = 128 and B = 128. XATTN_F32 runs plain FP32 CUDA-core kernels for small
  * problems and needs d in {32, 64, 128} and B <= 256.
