@@ -525,3 +525,86 @@ def test_short_last_block_batched_shapes():
     _, lists = O.select_blocks(P, [0.9, 1.0], True)
     Os, lse = O.sparse_attention(Q, K, V, 16, True, lists)
     assert Os.shape == (1, 2, 40, 4) and np.isfinite(Os).all() and np.isfinite(lse).all()
+
+
+# ------------------------------------------- batched wrappers (GQA, tau) ----
+def _gqa_inputs():
+    """hq = 4 query heads over hkv = 2 KV heads, batch 2, with K and V of each
+    KV head and batch entry drawn apart (V scaled so it can never pass for K)."""
+    b, hq, hkv, L, d = 2, 4, 2, 48, 4
+    Q = _rand(b, hq, L, d)
+    K = _rand(b, hkv, L, d)
+    V = _rand(b, hkv, L, d, scale=5.0)
+    K[:, 1] += 2.0
+    V[1] -= 3.0
+    return Q, K, V
+
+
+def _random_lists(b, hq, NB, causal):
+    lists = {}
+    for bb in range(b):
+        for h in range(hq):
+            for qb in range(NB):
+                n = qb + 1 if causal else NB
+                lists[(bb, h, qb)] = sorted({0} | {j for j in range(n) if rng.random() < 0.5})
+    return lists
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_batched_sparse_attention_reads_the_gqa_kv_head(causal):
+    """The batched attention wrapper gives query head h of batch entry bb the
+    keys and values of KV head h // (hq / hkv) of the same entry (GQA, the
+    mapping read into the pages). Pinned against the triple-loop attention on
+    hand-picked operands, so a K/V swap, the h % hkv mapping or a batch mix-up
+    in the wrapper fails here."""
+    Q, K, V = _gqa_inputs()
+    b, hq, L, _ = Q.shape
+    hkv, B = K.shape[1], 16
+    NB = L // B
+    lists = _random_lists(b, hq, NB, causal)
+    Os, lse = O.sparse_attention(Q, K, V, B, causal, lists)
+    for bb in range(b):
+        for h in range(hq):
+            kv = h // (hq // hkv)
+            want, _ = O.dense_attention_naive(
+                Q[bb, h], K[bb, kv], V[bb, kv], causal,
+                allowed=lambda i, j, bb=bb, h=h: (j // B) in lists[(bb, h, i // B)])
+            np.testing.assert_allclose(Os[bb, h], want, rtol=0, atol=1e-12)
+    # planted mistakes: each gives a different answer on these inputs
+    h = 1
+    for kk, vv in ((V[0, 0], K[0, 0]),             # K and V swapped
+                   (K[0, h % hkv], V[0, h % hkv]),  # h % hkv instead of h // g
+                   (K[1, 0], V[1, 0])):            # the other batch entry's KV head
+        wrong, _ = O.dense_attention_naive(
+            Q[0, h], kk, vv, causal,
+            allowed=lambda i, j: (j // B) in lists[(0, h, i // B)])
+        assert np.max(np.abs(wrong - Os[0, h])) > 1e-3
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_batched_select_uses_each_heads_tau(causal):
+    """The batched selection applies head h's own threshold tau[h] (per-head
+    tau, §2.3 of the pages; an input of the hot path). Every row is checked
+    against brute force over all subsets with that head's tau, and the rows
+    of heads 1..3 would differ under tau[0]."""
+    b, hq, NB = 2, 4, 7
+    taus = [0.5, 0.7, 0.85, 0.97]
+    P = np.zeros((b, hq, NB, NB))
+    for bb in range(b):
+        for h in range(hq):
+            for qb in range(NB):
+                n = qb + 1 if causal else NB
+                P[bb, h, qb, :n] = rng.dirichlet(np.ones(n) * 0.7)
+    mask, lists = O.select_blocks(P, taus, causal)
+    differs = 0
+    for bb in range(b):
+        for h in range(hq):
+            for qb in range(NB):
+                n = qb + 1 if causal else NB
+                row = list(P[bb, h, qb, :n])
+                want = sorted(_brute_minimal(row, taus[h]))
+                assert list(lists[(bb, h, qb)]) == want, (bb, h, qb)
+                assert list(np.nonzero(mask[bb, h, qb])[0]) == want
+                if h > 0 and sorted(_brute_minimal(row, taus[0])) != want:
+                    differs += 1
+    assert differs > 0   # tau[0] for every head would fail the rows above
