@@ -66,3 +66,39 @@ def test_sampler_falls_back_without_nvml(monkeypatch):
     monkeypatch.setitem(sys.modules, "pynvml", broken)
     bench = importlib.import_module("bench")
     assert isinstance(bench.clock_sampler(0), bench.ClockSampler)
+
+
+def test_peak_follows_the_clocks():
+    """Burst bf16 peak when the timed region ran at the maximum SM clock, the
+    sustained (power-capped) figure otherwise."""
+    bench = importlib.import_module("bench")
+    pk = {"bf16": 1694.7, "bf16_sustained": 1438.2, "source": "measured"}
+    peak, src = bench.bf16_peak_for_clocks(pk, {"sm_mhz": 1965, "sm_max_mhz": 1965})
+    assert peak == 1694.7 and "burst" in src
+    peak, src = bench.bf16_peak_for_clocks(pk, {"sm_mhz": 1514, "sm_max_mhz": 1965})
+    assert peak == 1438.2 and "sustained" in src
+    peak, _ = bench.bf16_peak_for_clocks(pk, {"sm_mhz": None, "sm_max_mhz": None})
+    assert peak == 1438.2
+
+
+def test_cpu_baseline_scales_setup_and_units_apart(monkeypatch):
+    """The oracle sample converts only the sampled heads, times the per-head
+    set-up apart from the per-block work, and scales each by its own count."""
+    import numpy as np
+    import torch
+    bench = importlib.import_module("bench")
+
+    class P:
+        pass
+    prob = P()
+    g = torch.Generator().manual_seed(0)
+    prob.batch, prob.hq, prob.hkv, prob.L, prob.d, prob.B, prob.S = 1, 4, 2, 256, 8, 32, 4
+    prob.NB, prob.causal = 8, True
+    prob.Q = torch.randn(1, 4, 256, 8, generator=g)
+    prob.K = torch.randn(1, 2, 256, 8, generator=g)
+    prob.V = torch.randn(1, 2, 256, 8, generator=g)
+    prob.tau = np.full(4, 0.9, np.float32)
+    cb = bench.oracle_sample(prob, [0, 3], n_blocks=4)
+    assert cb["kind"] == "oracle" and cb["unit"] == "ms/layer" and cb["extrapolated"]
+    assert cb["value"] > 0 and cb["measured_s"] > 0
+    assert "query heads [0, 3] of 4 x 4 of 8 query blocks" in cb["sample"]
