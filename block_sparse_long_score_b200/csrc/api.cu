@@ -27,15 +27,52 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
 
-// Looks up the device state of the current device, creating it on first use.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+std::mutex g_ctx_mu;
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+int current_context_id(unsigned long long* id) {
+  *id = 0;
+  {
+    std::lock_guard<std::mutex> lock(g_ctx_mu);
+    if (!g_ctx_get_current || !g_ctx_get_id) {
+      void* f1 = nullptr;
+      void* f2 = nullptr;
+      cudaDriverEntryPointQueryResult q1, q2;
+      if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) !=
+              cudaSuccess ||
+          q1 != cudaDriverEntryPointSuccess || !f1 ||
+          cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+          q2 != cudaDriverEntryPointSuccess || !f2)
+        return XATTN_ERR_CUDA;
+      g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+      g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f2);
+    }
+  }
+  CUcontext c = nullptr;
+  if (g_ctx_get_current(&c) != CUDA_SUCCESS) return XATTN_ERR_CUDA;
+  if (c == nullptr) return XATTN_OK;
+  return g_ctx_get_id(c, id) == CUDA_SUCCESS ? XATTN_OK : XATTN_ERR_CUDA;
+}
+
+// Looks up the device state of the current device, creating it on first use
+// and again whenever the device's context has changed since.
 int device_state(DeviceState** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return XATTN_ERR_CUDA;
+  unsigned long long ctx = 0;
+  int rc = current_context_id(&ctx);
+  if (rc != XATTN_OK) return rc;
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState& s = g_dev[dev];
-  if (!s.ready) {
+  if (!s.ready || ctx == 0 || s.ctx_id != ctx) {
+    s.ready = false;
     void* addr = nullptr;
+    // also makes the device's primary context current if there was none
     if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess) return XATTN_ERR_CUDA;
+    if ((rc = current_context_id(&ctx)) != XATTN_OK || ctx == 0) return XATTN_ERR_CUDA;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return XATTN_ERR_CUDA;
@@ -50,6 +87,7 @@ int device_state(DeviceState** out) {
     }
     s.status = static_cast<int*>(addr);
     s.num_sms = sms;
+    s.ctx_id = ctx;
     s.ready = true;
   }
   *out = &s;

@@ -14,11 +14,19 @@ constexpr int kMaxDevices = 64;
 
 struct DeviceState {
   bool ready = false;
-  int* status = nullptr;  // device address of the status word
+  unsigned long long ctx_id = 0;  // context the addresses below belong to
+  int* status = nullptr;          // device address of the status word
   int num_sms = 0;
 };
 
-// State of the current device, created on first use. Returns an xattn_status.
+// Process-unique ID of the current CUDA context (cuCtxGetId); 0 when the
+// thread has no current context yet. Device addresses of module variables
+// belong to one context: a cache keyed by this ID is rebuilt when the context
+// changes (for example after cudaDeviceReset and a new primary context).
+int current_context_id(unsigned long long* id);
+
+// State of the current device, created on first use and rebuilt when the
+// device's context changes. Returns an xattn_status.
 int device_state(DeviceState** out);
 // Checks a shape and fills the derived sizes. Returns an xattn_status.
 int check_shape(const xattn_shape* sh, Dims* D);

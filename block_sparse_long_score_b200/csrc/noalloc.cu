@@ -28,20 +28,29 @@ static __device__ __align__(256) unsigned long long g_noalloc_order[XATTN_NOALLO
 
 std::mutex g_scratch_mu;
 unsigned long long* g_scratch_ptr[host::kMaxDevices] = {};
+unsigned long long g_scratch_ctx[host::kMaxDevices] = {};  // context of each cached address
 
 // Device address of g_noalloc_order on the current device. In host code the
-// symbol itself is only a host-side stand-in, so the address is looked up
-// once per device with cudaGetSymbolAddress and cached.
+// symbol itself is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress, once per device and context, and cached. A new
+// context on the device (after cudaDeviceReset, say) holds the array at a new
+// address, so the cache is keyed by the context's process-unique ID.
 int scratch_address(unsigned long long** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= host::kMaxDevices)
     return XATTN_ERR_CUDA;
+  unsigned long long ctx = 0;
+  int rc = host::current_context_id(&ctx);
+  if (rc != XATTN_OK) return rc;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (g_scratch_ptr[dev] == nullptr || ctx == 0 || g_scratch_ctx[dev] != ctx) {
+    g_scratch_ptr[dev] = nullptr;
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_order) != cudaSuccess || p == nullptr)
       return XATTN_ERR_CUDA;
+    if ((rc = host::current_context_id(&ctx)) != XATTN_OK || ctx == 0) return XATTN_ERR_CUDA;
     g_scratch_ptr[dev] = static_cast<unsigned long long*>(p);
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return XATTN_OK;
@@ -61,16 +70,17 @@ extern "C" int xattn_sparse_attn_noalloc(const void* Q, const void* K, const voi
   int rc = check_shape(shape, &D);
   if (rc != XATTN_OK) return rc;
   if (!Q || !K || !V || !counts || !idx || !O) return XATTN_ERR_INVALID_ARG;
-  const long long units = static_cast<long long>(D.batch) * D.hq * D.NB;
-  if (units > XATTN_NOALLOC_MAX_UNITS) return XATTN_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (D.dtype != XATTN_BF16) {
-    // the fp32 kernel maps rows to warps directly and needs no scratch
+    // the fp32 kernel maps rows to warps directly and needs no scratch, so
+    // the unit limit does not apply to it
     return cuda_status(launch_attn_simt(D, static_cast<const float*>(Q),
                                         static_cast<const float*>(K),
                                         static_cast<const float*>(V), counts, idx,
                                         static_cast<float*>(O), lse, st));
   }
+  const long long units = static_cast<long long>(D.batch) * D.hq * D.NB;
+  if (units > XATTN_NOALLOC_MAX_UNITS) return XATTN_ERR_WORKSPACE;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
     return XATTN_ERR_INVALID_ARG;
   DeviceState* ds = nullptr;

@@ -137,6 +137,15 @@ def _shape_of(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal: bool) ->
     return make_shape(b, hq, K.shape[1], L, d, B, S, causal, Q.dtype)
 
 
+def _attn_shape(Q, K, V, counts, idx, B: int, causal: bool) -> _Shape:
+    """Shape of an attention call, after checking V against K and the block
+    lists against the number of work units."""
+    shape = _shape_of(Q, K, B, 1, causal)
+    _check_shape(V, K.shape, "V")
+    _check_lists(counts, idx, shape.batch, shape.hq, -(-shape.L // max(shape.B, 1)))
+    return shape
+
+
 def _check(t: torch.Tensor, name: str, dtype=None) -> None:
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
@@ -144,6 +153,33 @@ def _check(t: torch.Tensor, name: str, dtype=None) -> None:
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _check_shape(t: torch.Tensor, shape, name: str) -> None:
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _check_lists(counts: torch.Tensor, idx: torch.Tensor, batch: int, hq: int, NB: int) -> None:
+    """counts [batch, hq, NB] and idx [batch, hq, NB, NB] (the kernels index
+    them by unit; a smaller buffer would be read past its end)."""
+    if counts.numel() != batch * hq * NB or idx.numel() != batch * hq * NB * NB:
+        raise ValueError(f"counts / idx must hold {batch}x{hq}x{NB} rows of {NB} entries, got "
+                         f"{tuple(counts.shape)} / {tuple(idx.shape)}")
+
+
+def _check_select_outputs(mask, counts, idx, batch: int, hq: int, NB: int) -> None:
+    for t, n in ((mask, "mask"), (counts, "counts"), (idx, "idx")):
+        _check(t, n, torch.int32)
+    _check_shape(mask, (batch, hq, NB, (NB + 31) // 32), "mask")
+    _check_shape(counts, (batch, hq, NB), "counts")
+    _check_shape(idx, (batch, hq, NB, NB), "idx")
+
+
+def _same_device(ref: torch.Tensor, *ts) -> None:
+    for t in ts:
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"every tensor must be on {ref.device}, got one on {t.device}")
 
 
 def _stream(device) -> ctypes.c_void_p:
@@ -189,10 +225,17 @@ def xattn_score(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal: bool,
     if probs is None:
         probs = torch.empty(shape.batch, shape.hq, NB, NB, device=Q.device, dtype=torch.float32)
     _check(probs, "probs", torch.float32)
+    _check_shape(probs, (shape.batch, shape.hq, NB, NB), "probs")
     need = xattn_score_workspace_bytes(shape)
     if workspace is None:
         workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
     _check(workspace, "workspace")
+    _same_device(Q, K, probs, workspace)
+    with torch.cuda.device(Q.device):
+        return _score_call(Q, K, S, shape, probs, workspace, perm)
+
+
+def _score_call(Q, K, S, shape, probs, workspace, perm):
     if perm is None:
         rc = _lib().xattn_score(Q.data_ptr(), K.data_ptr(), ctypes.byref(shape),
                                 probs.data_ptr(), workspace.data_ptr(),
@@ -231,8 +274,8 @@ def _select_outputs(probs: torch.Tensor, causal: bool, out: Optional[tuple]):
         idx = torch.empty(b, hq, NB, NB, device=probs.device, dtype=torch.int32)
     else:
         mask, counts, idx = out
-    for t, n in ((mask, "mask"), (counts, "counts"), (idx, "idx")):
-        _check(t, n, torch.int32)
+    _check_select_outputs(mask, counts, idx, b, hq, NB)
+    _same_device(probs, mask, counts, idx)
     return shape, mask, counts, idx
 
 
@@ -250,8 +293,9 @@ def xattn_select(probs: torch.Tensor, tau: Sequence[float], causal: bool,
     shape, mask, counts, idx = _select_outputs(probs, causal, out)
     taus = _per_head(tau, shape.hq, "tau", float)
     tarr = (ctypes.c_float * shape.hq)(*taus)
-    rc = _lib().xattn_select(probs.data_ptr(), tarr, ctypes.byref(shape), mask.data_ptr(),
-                             counts.data_ptr(), idx.data_ptr(), _stream(probs.device))
+    with torch.cuda.device(probs.device):
+        rc = _lib().xattn_select(probs.data_ptr(), tarr, ctypes.byref(shape), mask.data_ptr(),
+                                 counts.data_ptr(), idx.data_ptr(), _stream(probs.device))
     _raise("xattn_select", rc)
     return mask, counts, idx
 
@@ -270,6 +314,7 @@ def xattn_score_select(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal:
         probs = torch.empty(shape.batch, shape.hq, NB, NB, device=Q.device, dtype=torch.float32)
     if want_p:
         _check(probs, "probs", torch.float32)
+        _check_shape(probs, (shape.batch, shape.hq, NB, NB), "probs")
     W = (NB + 31) // 32
     if out is None:
         mask = torch.empty(shape.batch, shape.hq, NB, W, device=Q.device, dtype=torch.int32)
@@ -277,19 +322,20 @@ def xattn_score_select(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal:
         idx = torch.empty(shape.batch, shape.hq, NB, NB, device=Q.device, dtype=torch.int32)
     else:
         mask, counts, idx = out
-    for t, n in ((mask, "mask"), (counts, "counts"), (idx, "idx")):
-        _check(t, n, torch.int32)
+    _check_select_outputs(mask, counts, idx, shape.batch, shape.hq, NB)
     taus = _per_head(tau, shape.hq, "tau", float)
     tarr = (ctypes.c_float * shape.hq)(*taus)
     need = xattn_score_workspace_bytes(shape)
     if workspace is None:
         workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
     _check(workspace, "workspace")
-    rc = _lib().xattn_score_select(Q.data_ptr(), K.data_ptr(), ctypes.byref(shape), tarr,
-                                   probs.data_ptr() if want_p else None, mask.data_ptr(),
-                                   counts.data_ptr(), idx.data_ptr(), workspace.data_ptr(),
-                                   workspace.numel() * workspace.element_size(),
-                                   _stream(Q.device))
+    _same_device(Q, K, probs if want_p else None, mask, counts, idx, workspace)
+    with torch.cuda.device(Q.device):
+            rc = _lib().xattn_score_select(Q.data_ptr(), K.data_ptr(), ctypes.byref(shape), tarr,
+                                       probs.data_ptr() if want_p else None, mask.data_ptr(),
+                                       counts.data_ptr(), idx.data_ptr(), workspace.data_ptr(),
+                                       workspace.numel() * workspace.element_size(),
+                                       _stream(Q.device))
     _raise("xattn_score_select", rc)
     return (probs, mask, counts, idx) if want_p else (mask, counts, idx)
 
@@ -300,8 +346,10 @@ def xattn_select_topk(probs: torch.Tensor, k: Sequence[int], causal: bool,
     shape, mask, counts, idx = _select_outputs(probs, causal, out)
     ks = _per_head(k, shape.hq, "k", int)
     karr = (ctypes.c_int32 * shape.hq)(*ks)
-    rc = _lib().xattn_select_topk(probs.data_ptr(), karr, ctypes.byref(shape), mask.data_ptr(),
-                                  counts.data_ptr(), idx.data_ptr(), _stream(probs.device))
+    with torch.cuda.device(probs.device):
+        rc = _lib().xattn_select_topk(probs.data_ptr(), karr, ctypes.byref(shape),
+                                      mask.data_ptr(), counts.data_ptr(), idx.data_ptr(),
+                                      _stream(probs.device))
     _raise("xattn_select_topk", rc)
     return mask, counts, idx
 
@@ -312,9 +360,10 @@ def xattn_select_topratio(probs: torch.Tensor, ratio: Sequence[float], causal: b
     shape, mask, counts, idx = _select_outputs(probs, causal, out)
     rs = _per_head(ratio, shape.hq, "ratio", float)
     rarr = (ctypes.c_float * shape.hq)(*rs)
-    rc = _lib().xattn_select_topratio(probs.data_ptr(), rarr, ctypes.byref(shape),
-                                      mask.data_ptr(), counts.data_ptr(), idx.data_ptr(),
-                                      _stream(probs.device))
+    with torch.cuda.device(probs.device):
+        rc = _lib().xattn_select_topratio(probs.data_ptr(), rarr, ctypes.byref(shape),
+                                          mask.data_ptr(), counts.data_ptr(), idx.data_ptr(),
+                                          _stream(probs.device))
     _raise("xattn_select_topratio", rc)
     return mask, counts, idx
 
@@ -330,24 +379,29 @@ def xattn_sparse_attn(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, counts:
     _check(V, "V", Q.dtype)
     _check(counts, "counts", torch.int32)
     _check(idx, "idx", torch.int32)
-    shape = _shape_of(Q, K, B, 1, causal)
+    shape = _attn_shape(Q, K, V, counts, idx, B, causal)
     if out is None:
         out = torch.empty_like(Q)
     _check(out, "O", Q.dtype)
+    _check_shape(out, Q.shape, "O")
     want_lse = lse is not None and lse is not False
     if lse is True:
         lse = torch.empty(Q.shape[:3], device=Q.device, dtype=torch.float32)
     if want_lse:
         _check(lse, "lse", torch.float32)
+        _check_shape(lse, Q.shape[:3], "lse")
     need = xattn_attn_workspace_bytes(shape)
     if workspace is None:
         workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
     _check(workspace, "workspace")
-    rc = _lib().xattn_sparse_attn(Q.data_ptr(), K.data_ptr(), V.data_ptr(), ctypes.byref(shape),
-                                  counts.data_ptr(), idx.data_ptr(), out.data_ptr(),
-                                  lse.data_ptr() if want_lse else None, workspace.data_ptr(),
-                                  workspace.numel() * workspace.element_size(),
-                                  _stream(Q.device))
+    _same_device(Q, K, V, counts, idx, out, lse if want_lse else None, workspace)
+    with torch.cuda.device(Q.device):
+        rc = _lib().xattn_sparse_attn(Q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                      ctypes.byref(shape), counts.data_ptr(), idx.data_ptr(),
+                                      out.data_ptr(), lse.data_ptr() if want_lse else None,
+                                      workspace.data_ptr(),
+                                      workspace.numel() * workspace.element_size(),
+                                      _stream(Q.device))
     _raise("xattn_sparse_attn", rc)
     return (out, lse) if want_lse else out
 
@@ -364,14 +418,18 @@ def xattn_sparse_attn_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
     _check(counts, "counts", torch.int32)
     _check(idx, "idx", torch.int32)
     _check(out, "O", Q.dtype)
+    shape = _attn_shape(Q, K, V, counts, idx, B, causal)
+    _check_shape(out, Q.shape, "O")
     if lse is not None:
         _check(lse, "lse", torch.float32)
-    shape = _shape_of(Q, K, B, 1, causal)
-    rc = _lib().xattn_sparse_attn_noalloc(Q.data_ptr(), K.data_ptr(), V.data_ptr(),
-                                          ctypes.byref(shape), counts.data_ptr(),
-                                          idx.data_ptr(), out.data_ptr(),
-                                          lse.data_ptr() if lse is not None else None,
-                                          _stream(Q.device))
+        _check_shape(lse, Q.shape[:3], "lse")
+    _same_device(Q, K, V, counts, idx, out, lse)
+    with torch.cuda.device(Q.device):
+        rc = _lib().xattn_sparse_attn_noalloc(Q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                              ctypes.byref(shape), counts.data_ptr(),
+                                              idx.data_ptr(), out.data_ptr(),
+                                              lse.data_ptr() if lse is not None else None,
+                                              _stream(Q.device))
     _raise("xattn_sparse_attn_noalloc", rc)
     return out
 
@@ -393,8 +451,10 @@ def xattn_check_lists(Q: torch.Tensor, K: torch.Tensor, counts: torch.Tensor, id
     if bad is None:
         bad = torch.empty(1, device=Q.device, dtype=torch.int32)
     _check(bad, "bad", torch.int32)
-    rc = _lib().xattn_check_lists(counts.data_ptr(), idx.data_ptr(), ctypes.byref(shape),
-                                  bad.data_ptr(), _stream(Q.device))
+    _same_device(Q, counts, idx, bad)
+    with torch.cuda.device(Q.device):
+        rc = _lib().xattn_check_lists(counts.data_ptr(), idx.data_ptr(), ctypes.byref(shape),
+                                      bad.data_ptr(), _stream(Q.device))
     _raise("xattn_check_lists", rc)
     return bad
 
@@ -431,12 +491,15 @@ def xattn_prefill_host(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, B: int
         out = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=not Q.is_cuda,
                           device=Q.device)
     _check_any(out, "O", Q.dtype)
+    _check_shape(V, K.shape, "V")
+    _check_shape(out, Q.shape, "O")
     want_lse = lse is not None and lse is not False
     if lse is True:
         lse = torch.empty(Q.shape[:3], dtype=torch.float32, pin_memory=not Q.is_cuda,
                           device=Q.device)
     if want_lse:
         _check_any(lse, "lse", torch.float32)
+        _check_shape(lse, Q.shape[:3], "lse")
     taus = _per_head(tau, shape.hq, "tau", float)
     tarr = (ctypes.c_float * shape.hq)(*taus)
     need = xattn_prefill_host_workspace_bytes(shape, kv_heads_per_chunk)
@@ -478,11 +541,13 @@ def xattn_prefill_varlen(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
     if out is None:
         out = torch.empty_like(Q)
     _check(out, "O", Q.dtype)
+    _check_shape(out, Q.shape, "O")
     want_lse = lse is not None and lse is not False
     if lse is True:
         lse = torch.empty(hq * T, device=Q.device, dtype=torch.float32)
     if want_lse:
         _check(lse, "lse", torch.float32)
+        _check_shape(lse, (hq * T,), "lse")
     taus = _per_head(tau, hq, "tau", float)
     tarr = (ctypes.c_float * hq)(*taus)
     larr = (ctypes.c_int32 * len(lens))(*lens)
@@ -490,11 +555,14 @@ def xattn_prefill_varlen(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
     if workspace is None:
         workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
     _check(workspace, "workspace")
-    rc = _lib().xattn_prefill_varlen(Q.data_ptr(), K.data_ptr(), V.data_ptr(),
-                                     ctypes.byref(shape), len(lens), larr, tarr, out.data_ptr(),
-                                     lse.data_ptr() if want_lse else None, workspace.data_ptr(),
-                                     workspace.numel() * workspace.element_size(),
-                                     _stream(Q.device))
+    _same_device(Q, K, V, out, lse if want_lse else None, workspace)
+    with torch.cuda.device(Q.device):
+        rc = _lib().xattn_prefill_varlen(Q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                         ctypes.byref(shape), len(lens), larr, tarr,
+                                         out.data_ptr(), lse.data_ptr() if want_lse else None,
+                                         workspace.data_ptr(),
+                                         workspace.numel() * workspace.element_size(),
+                                         _stream(Q.device))
     _raise("xattn_prefill_varlen", rc)
     return (out, lse) if want_lse else out
 

@@ -221,7 +221,8 @@ int xattn_sparse_attn(const void* Q, const void* K, const void* V, const xattn_s
                       const int32_t* counts, const int32_t* idx, void* O, float* lse,
                       void* ws, size_t ws_bytes, void* stream);
 
-/* Largest batch*hq*NB accepted by xattn_sparse_attn_noalloc. */
+/* Largest batch*hq*NB accepted by xattn_sparse_attn_noalloc (bf16 calls; the
+ * fp32 kernel uses no scratch and has no such limit). */
 #define XATTN_NOALLOC_MAX_UNITS (1 << 18)
 
 /*
@@ -235,14 +236,16 @@ int xattn_sparse_attn(const void* Q, const void* K, const void* V, const xattn_s
  *
  * The work order lives in a __device__ array of the library, sized for
  * XATTN_NOALLOC_MAX_UNITS work units (2 MiB). Each GPU that loads the library
- * holds it until the process exits. Returns XATTN_ERR_WORKSPACE when
- * batch*hq*NB exceeds that limit.
+ * holds it until the process exits. A bf16 call returns XATTN_ERR_WORKSPACE
+ * when batch*hq*NB exceeds that limit (the fp32 path uses no scratch).
  *
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) and caches it; make that first call before any
- * stream capture. All calls on a device share the array and it keeps the last
- * call's contents. Calls whose kernels overlap on the GPU (for example on two
- * unordered streams) race on it, so order such calls on one stream.
+ * The first call on a device (and the first after the device's context has
+ * changed, e.g. after cudaDeviceReset) looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it for that context; make that first call
+ * before any stream capture. All calls on a device share the array and it
+ * keeps the last call's contents. Calls whose kernels overlap on the GPU (for
+ * example on two unordered streams) race on it, so order such calls on one
+ * stream.
  * Arguments and other errors are as for xattn_sparse_attn.
  */
 int xattn_sparse_attn_noalloc(const void* Q, const void* K, const void* V,

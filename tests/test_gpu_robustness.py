@@ -105,3 +105,40 @@ def test_canary_every_output_written(causal_case):
                 assert np.all(ixn[0, h, qb, n:] == SENT)   # nothing written past the count
     assert torch.all(torch.isfinite(out.float()))   # every row of O written
     assert torch.all(torch.isfinite(lse))           # every row has a visible key here
+
+
+def test_binding_rejects_buffers_of_the_wrong_shape():
+    """The binding checks every caller-passed buffer against the shape before
+    the call: a buffer too small for what the kernels write or read raises
+    here instead of reaching the GPU."""
+    from block_sparse_long_score_b200 import xattn_sparse_attn_noalloc
+    prob, Q, K, V = _small()
+    taus = prob.tau.tolist()
+    P = xattn_score(Q, K, prob.B, prob.S, prob.causal)
+    mask, counts, idx = xattn_select(P, taus, prob.causal)
+    torch.cuda.synchronize()
+    bad_calls = [
+        lambda: xattn_sparse_attn(Q, K, V[:, :, :-128], counts, idx, prob.B, prob.causal),
+        lambda: xattn_sparse_attn(Q, K, V, counts[..., :-1], idx, prob.B, prob.causal),
+        lambda: xattn_sparse_attn(Q, K, V, counts, idx[..., :-1], prob.B, prob.causal),
+        lambda: xattn_sparse_attn(Q, K, V, counts, idx, prob.B, prob.causal,
+                                  out=torch.empty_like(Q)[:, :, :-1]),
+        lambda: xattn_sparse_attn(Q, K, V, counts, idx, prob.B, prob.causal,
+                                  lse=torch.empty(Q.shape[:2], device=DEV)),
+        lambda: xattn_sparse_attn_noalloc(Q, K, V, counts, idx, prob.B, prob.causal,
+                                          torch.empty_like(Q)[:, :1]),
+        lambda: xattn_sparse_attn_noalloc(Q, K, V, counts, idx, prob.B, prob.causal,
+                                          torch.empty_like(Q),
+                                          torch.empty(Q.shape[:3][:-1] + (7,), device=DEV)),
+        lambda: xattn_sparse_attn_noalloc(Q, K, V[:, :, :-128], counts, idx, prob.B,
+                                          prob.causal, torch.empty_like(Q)),
+        lambda: xattn_score(Q, K, prob.B, prob.S, prob.causal, probs=P[..., :-1]),
+        lambda: xattn_select(P, taus, prob.causal, out=(mask[..., :-1], counts, idx)),
+        lambda: xattn_score_select(Q, K, prob.B, prob.S, prob.causal, taus,
+                                   out=(mask, counts[:, :1], idx)),
+    ]
+    for i, call in enumerate(bad_calls):
+        with pytest.raises(ValueError):
+            call()
+            pytest.fail(f"bad call {i} was accepted")
+    assert xattn_get_device_status() == 0
