@@ -71,6 +71,15 @@ def bf16_peak_for_clocks(pk: dict, clk: dict) -> tuple:
     return pk["bf16_sustained"], f"{pk['source']} bf16 sustained ({seen} in the timed region)"
 
 
+def split_config(args, world: int, hq: int, hkv: int) -> dict:
+    """How the ranks share the work: whole-layer replicas, or one layer cut
+    into contiguous KV-head ranges (the config's hq/hkv are then this rank's)."""
+    if world > 1 and args.split == "heads":
+        return {"parallelism": f"heads{world}", "layer_hq": hq, "layer_hkv": hkv,
+                "gather_O": bool(args.gather)}
+    return {"parallelism": f"replicas{world}" if world > 1 else "replicas"}
+
+
 def workload_config(prob) -> dict:
     kinds = {"c1": "llama3.1-8b attention layer", "c2": "llama3.1-8b attention layer",
              "c3": "llama3.1-8b attention layer", "c4": "video-DiT attention layer (30x2560)"}
@@ -99,10 +108,29 @@ def max_over_ranks(x: float, device=None) -> float:
     return float(t.item())
 
 
-def whole_job_ms_per_layer(ms_step_max: float, world: int) -> float:
+def whole_job_ms_per_layer(ms_step_max: float, world: int, split: str = "replicas") -> float:
     """Replicas: every rank runs one layer per step, so the whole job finishes
-    `world` layers per (slowest rank's) step."""
-    return ms_step_max / world
+    `world` layers per (slowest rank's) step. Head split: the ranks share one
+    layer per step, so a layer takes the slowest rank's step."""
+    return ms_step_max if split == "heads" else ms_step_max / world
+
+
+def local_heads(prob, rank: int, world: int):
+    """The problem restricted to this rank's KV heads (and their query heads)
+    for the head-sharded split: the same layer, cut by KV-head groups."""
+    import copy
+    from block_sparse_long_score_b200.shard import kv_head_range
+    kv0, kv1 = kv_head_range(rank, world, prob.hkv)
+    if kv1 <= kv0:
+        raise ValueError(f"rank {rank} of {world} has no KV head of {prob.hkv}")
+    g = prob.hq // prob.hkv
+    loc = copy.copy(prob)
+    loc.Q = prob.Q[:, kv0 * g:kv1 * g].contiguous()
+    loc.K = prob.K[:, kv0:kv1].contiguous()
+    loc.V = prob.V[:, kv0:kv1].contiguous()
+    loc.tau = prob.tau[kv0 * g:kv1 * g].copy()
+    loc.hq, loc.hkv = (kv1 - kv0) * g, kv1 - kv0
+    return loc
 
 
 def dense_equiv_flops(prob) -> float:
@@ -317,6 +345,9 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     prob = make_problem(args.config, **problem_overrides(args))
+    layer_hq, layer_hkv = prob.hq, prob.hkv
+    if args.split == "heads" and world > 1:
+        prob = local_heads(prob, rank, world)
     Qh, Kh, Vh = prob.Q.pin_memory(), prob.K.pin_memory(), prob.V.pin_memory()
     Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
     shape = make_shape(prob.batch, prob.hq, prob.hkv, prob.L, prob.d, prob.B, prob.S,
@@ -331,6 +362,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     idx = torch.empty(prob.batch, prob.hq, NB, NB, device=dev, dtype=torch.int32)
     out = torch.empty_like(Q)
     taus = prob.tau.tolist()
+    tau_d = torch.tensor(taus, dtype=torch.float32, device=dev)   # per-head tau, device-resident
     stream = torch.cuda.current_stream(dev)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
@@ -341,7 +373,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
         if args.fused:
             # scoring, block sums and find_blocks in one call (P stays on chip);
             # its time is reported under "score", "select" is 0
-            xattn_score_select(Q, K, prob.B, prob.S, prob.causal, taus,
+            xattn_score_select(Q, K, prob.B, prob.S, prob.causal, tau_d,
                                out=(mask, counts, idx), workspace=ws_s)
             if ev:
                 ev[1].record(stream)
@@ -349,13 +381,18 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
             xattn_score(Q, K, prob.B, prob.S, prob.causal, probs=probs, workspace=ws_s)
             if ev:
                 ev[1].record(stream)
-            xattn_select(probs, taus, prob.causal, out=(mask, counts, idx))
+            xattn_select(probs, tau_d, prob.causal, out=(mask, counts, idx))
         if ev:
             ev[2].record(stream)
         xattn_sparse_attn(Q, K, V, counts, idx, prob.B, prob.causal, out=out, workspace=ws_a)
+        if gather:
+            # the whole layer's O on every rank (NCCL all-gather of the head ranges)
+            from block_sparse_long_score_b200.shard import gather_heads
+            gather_heads(out, layer_hq, layer_hkv)
         if ev:
             ev[3].record(stream)
 
+    gather = args.split == "heads" and args.gather and world > 1
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -457,7 +494,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     if not args.no_dense:
         if args.fused:
             probs.zero_()   # the fused path never wrote P; tau = 1 selects all either way
-        xattn_select(probs, [1.0] * prob.hq, prob.causal, out=(mask, counts, idx))
+        xattn_select(probs, torch.ones_like(tau_d), prob.causal, out=(mask, counts, idx))
         xattn_sparse_attn(Q, K, V, counts, idx, prob.B, prob.causal, out=out, workspace=ws_a)
         torch.cuda.synchronize(dev)
         d0 = torch.cuda.Event(enable_timing=True)
@@ -497,18 +534,18 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     traffic = None if (args.heads or args.fused) else TRAFFIC_BYTES.get((args.config, dom))
     line = {
         "metric": METRIC,
-        "value": whole_job_ms_per_layer(ms_step, world),
+        "value": whole_job_ms_per_layer(ms_step, world, args.split),
         "unit": "ms/layer",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": ms_step,
         "higher_is_better": False,
-        "scaling": "weak",
+        "scaling": "strong" if args.split == "heads" and world > 1 else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded Llama-3.1-8B-shaped Q/K/V with planted sinks and slash bands)",
-        "config": dict(workload_config(prob),
+        "config": dict(workload_config(prob), **split_config(args, world, layer_hq, layer_hkv),
                        path="xattn_score_select + xattn_sparse_attn" if args.fused
                        else "xattn_score + xattn_select + xattn_sparse_attn"),
         "dense_equiv_tflops": dense_tflops,
@@ -540,7 +577,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
             "peak_source": peak_source,
         },
         "e2e": {
-            "value": whole_job_ms_per_layer(e2e_ms, world),
+            "value": whole_job_ms_per_layer(e2e_ms, world, args.split),
             "unit": "ms/layer",
             "h2d_bytes_per_step": int(Q.numel() * 2 + K.numel() * 2 + V.numel() * 2),
             "d2h_bytes_per_step": int(out.numel() * 2),
@@ -548,7 +585,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
                     "compute, one KV head per chunk)",
         },
         # the same copies and calls one after another on one stream, for context
-        "e2e_serial": {"value": whole_job_ms_per_layer(e2e_serial_ms, world),
+        "e2e_serial": {"value": whole_job_ms_per_layer(e2e_serial_ms, world, args.split),
                        "unit": "ms/layer"},
         "gpu_launches": (4 if args.fused else 6) * args.steps,
         "clocks": clk,
@@ -626,6 +663,11 @@ def main() -> None:
     ap.add_argument("--stride", type=int, default=0, help="stride S for the video layer (c4)")
     ap.add_argument("--fused", action="store_true",
                     help="run scoring and selection as one call (xattn_score_select)")
+    ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
+                    help="multi-GPU: whole-layer replicas (default) or one layer cut into "
+                         "contiguous KV-head ranges, one per rank")
+    ap.add_argument("--gather", action="store_true",
+                    help="with --split heads: all-gather O (NCCL) inside every step")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling case: keep this many query heads (default: all 32)")
     args = ap.parse_args()

@@ -250,6 +250,32 @@ int tau_arg(const float* tau, int hq, TauArg* ta) {
   return XATTN_OK;
 }
 
+// Per-head thresholds read by the kernels from a device array; each kernel
+// checks its head's value and reports one outside (0, 1] in the status word.
+void tau_dev_arg(const float* tau_dev, int* status, TauArg* ta) {
+  std::memset(ta, 0, sizeof(*ta));
+  ta->dev = tau_dev;
+  ta->status = status;
+}
+
+// Scoring, then the fused reduce + find_blocks, with validated thresholds.
+int score_select_impl(const void* Q, const void* K, const xattn_shape* shape, const TauArg& ta,
+                      float* probs, uint32_t* mask, int32_t* counts, int32_t* idx, void* ws,
+                      size_t ws_bytes, void* stream) {
+  Dims D;
+  int rc = check_score_args(Q, K, shape, ws, ws_bytes, &D);
+  if (rc != XATTN_OK) return rc;
+  if (!mask || !counts || !idx) return XATTN_ERR_INVALID_ARG;
+  if (D.S > 256) return XATTN_ERR_UNSUPPORTED;  // S divides B <= 256 for every valid shape
+  PermArg perm;  // the antidiagonal
+  std::memset(&perm, 0, sizeof(perm));
+  for (int i = 0; i < D.S; ++i) perm.q[i] = static_cast<uint8_t>(D.S - 1 - i);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* part = static_cast<float*>(ws);
+  if ((rc = score_partials(Q, K, D, perm, part, st)) != XATTN_OK) return rc;
+  return cuda_status(launch_score_select(D, part, probs, ta, mask, counts, idx, st));
+}
+
 // Fixed-budget selection (arguments already validated into `budget`).
 int select_budget_impl(const float* probs, const BudgetArg& budget, const Dims& D,
                        uint32_t* mask, int32_t* counts, int32_t* idx, void* stream) {
@@ -302,10 +328,10 @@ int xattn_select(const float* probs, const float* tau, const xattn_shape* shape,
   int rc = check_shape(shape, &D);
   if (rc != XATTN_OK) return rc;
   if (!probs || !tau || !mask || !counts || !idx) return XATTN_ERR_INVALID_ARG;
-  TauArg ta;
-  if ((rc = tau_arg(tau, D.hq, &ta)) != XATTN_OK) return rc;
   DeviceState* ds = nullptr;
   if ((rc = device_state(&ds)) != XATTN_OK) return rc;
+  TauArg ta;
+  tau_dev_arg(tau, ds->status, &ta);
   return cuda_status(
       launch_select(D, probs, ta, mask, counts, idx, ds->num_sms, static_cast<cudaStream_t>(stream)));
 }
@@ -314,20 +340,36 @@ int xattn_score_select(const void* Q, const void* K, const xattn_shape* shape, c
                        float* probs, uint32_t* mask, int32_t* counts, int32_t* idx, void* ws,
                        size_t ws_bytes, void* stream) {
   Dims D;
-  int rc = check_score_args(Q, K, shape, ws, ws_bytes, &D);
+  int rc = check_score_args(Q, K, shape, ws, ws_bytes, &D);  // every host check first
   if (rc != XATTN_OK) return rc;
   if (!tau || !mask || !counts || !idx) return XATTN_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(&ds)) != XATTN_OK) return rc;
   TauArg ta;
-  if ((rc = tau_arg(tau, D.hq, &ta)) != XATTN_OK) return rc;
-  if (D.S > 256) return XATTN_ERR_UNSUPPORTED;  // S divides B <= 256 for every valid shape
-  PermArg perm;  // the antidiagonal
-  std::memset(&perm, 0, sizeof(perm));
-  for (int i = 0; i < D.S; ++i) perm.q[i] = static_cast<uint8_t>(D.S - 1 - i);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* part = static_cast<float*>(ws);
-  if ((rc = score_partials(Q, K, D, perm, part, st)) != XATTN_OK) return rc;
-  return cuda_status(launch_score_select(D, part, probs, ta, mask, counts, idx, st));
+  tau_dev_arg(tau, ds->status, &ta);
+  return score_select_impl(Q, K, shape, ta, probs, mask, counts, idx, ws, ws_bytes, stream);
 }
+
+}  // extern "C"
+
+namespace xattn {
+namespace host {
+
+int score_select_host_tau(const void* Q, const void* K, const xattn_shape* shape,
+                          const float* tau_host, float* probs, uint32_t* mask, int32_t* counts,
+                          int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+  if (!tau_host || !shape) return XATTN_ERR_INVALID_ARG;
+  if (shape->hq < 1 || shape->hq > XATTN_MAX_HEADS) return XATTN_ERR_INVALID_ARG;
+  TauArg ta;
+  const int rc = tau_arg(tau_host, shape->hq, &ta);
+  if (rc != XATTN_OK) return rc;
+  return score_select_impl(Q, K, shape, ta, probs, mask, counts, idx, ws, ws_bytes, stream);
+}
+
+}  // namespace host
+}  // namespace xattn
+
+extern "C" {
 
 int xattn_select_topk(const float* probs, const int32_t* k, const xattn_shape* shape,
                       uint32_t* mask, int32_t* counts, int32_t* idx, void* stream) {
@@ -422,7 +464,9 @@ int xattn_get_device_status(void* stream) {
     if (cudaMemcpy(ds->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
       return XATTN_ERR_CUDA;
   }
-  return v == kStatusTimeout ? XATTN_ERR_TIMEOUT : XATTN_OK;
+  if (v == kStatusTimeout) return XATTN_ERR_TIMEOUT;
+  if (v == kStatusBadTau) return XATTN_ERR_INVALID_ARG;
+  return XATTN_OK;
 }
 
 const char* xattn_strerror(int status) {

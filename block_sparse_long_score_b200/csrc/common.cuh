@@ -13,6 +13,7 @@ namespace xattn {
 
 // Device status codes written into the per-device status word.
 constexpr int kStatusTimeout = 1;
+constexpr int kStatusBadTau = 2;  // a device-resident tau was outside (0, 1] (or NaN)
 
 struct Dims {
   int batch, hq, hkv, L, d, B, S, causal, dtype;
@@ -80,9 +81,26 @@ cudaError_t launch_score_simt(const Dims& D, const float* Q, const float* K,
 cudaError_t launch_score_reduce(const Dims& D, const float* part, float* probs,
                                 cudaStream_t st);
 
+// Per-head thresholds: read from the device array `dev` when it is set (the
+// C ABI's xattn_select / xattn_score_select), else taken from `v` (calls that
+// receive tau in host memory and pass it by value). A device value outside
+// (0, 1] is reported through `status` (kStatusBadTau) and its head's rows
+// select nothing.
 struct TauArg {
   float v[XATTN_MAX_HEADS];
+  const float* dev;
+  int* status;
 };
+
+// tau of query head h, or a negative value when a device-resident tau is
+// invalid (the caller then selects nothing and the status word records it).
+__device__ __forceinline__ double tau_of(const TauArg& tau, int h) {
+  if (tau.dev == nullptr) return static_cast<double>(tau.v[h]);
+  const float t = __ldg(tau.dev + h);
+  if (t > 0.0f && t <= 1.0f) return static_cast<double>(t);  // false for NaN
+  atomicExch(tau.status, kStatusBadTau);
+  return -1.0;
+}
 
 // find_blocks on every row of P (a register-only walk of the ranking, then
 // the histogram search on the rows it leaves; num_sms sizes that second grid).

@@ -31,6 +31,12 @@ int device_state(DeviceState** out);
 // Checks a shape and fills the derived sizes. Returns an xattn_status.
 int check_shape(const xattn_shape* sh, Dims* D);
 bool aligned16(const void* p);
+// xattn_score_select with the thresholds in HOST memory (checked on the host
+// and passed to the kernels by value), for the whole-step calls that take
+// tau from the host.
+int score_select_host_tau(const void* Q, const void* K, const xattn_shape* shape,
+                          const float* tau_host, float* probs, uint32_t* mask, int32_t* counts,
+                          int32_t* idx, void* ws, size_t ws_bytes, void* stream);
 // 2-D bf16 view [rows, 128] with 64 x 128 boxes and 128-byte swizzle.
 int make_map_2d(CUtensorMap* m, const void* ptr, long long rows);
 int cuda_status(cudaError_t e);

@@ -214,8 +214,8 @@ int xattn_prefill_host(const void* Q, const void* K, const void* V, const xattn_
       rc = XATTN_ERR_CUDA;
       break;
     }
-    rc = xattn_score_select(q_d[slot], k_d[slot], &cs, tau + hq0, nullptr, mask, counts, idx,
-                            score_ws, Lo.score_ws, st);
+    rc = score_select_host_tau(q_d[slot], k_d[slot], &cs, tau + hq0, nullptr, mask, counts,
+                               idx, score_ws, Lo.score_ws, st);
     if (rc != XATTN_OK) break;
     rc = xattn_sparse_attn(q_d[slot], k_d[slot], v_d[slot], &cs, counts, idx, o_d[slot],
                            lse ? lse_d[slot] : nullptr, attn_ws, Lo.attn_ws, st);

@@ -6,12 +6,14 @@
 // partials to the row of P (the same arithmetic as the reduce kernel, so P is
 // bit-identical to xattn_score's) and stage it in shared memory; P goes to
 // HBM only if the caller asks for it. Warp 0 then finds the find_blocks cut of
-// the staged row (the search of the selection kernel) and writes the mask,
-// the count and the ascending index list; the other warps are done. Compared
+// the staged row (the selection kernel's threshold filter, and its histogram
+// search for a row the filter leaves) and writes the mask, the count and the
+// ascending index list; the other warps are done. Compared
 // with xattn_score followed by xattn_select this saves P's write and re-read
 // and one launch.
 #include "reduce_core.cuh"
 #include "select_core.cuh"
+#include "select_filter.cuh"
 
 namespace xattn {
 namespace {
@@ -25,7 +27,9 @@ __global__ void __launch_bounds__(kThreads)
                         int32_t* __restrict__ idx) {
   extern __shared__ __align__(16) uint8_t smem[];
   sel::WarpSmem& W = *reinterpret_cast<sel::WarpSmem*>(smem);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + sizeof(sel::WarpSmem));  // nb_stage
+  filt::WarpBuf& FB = *reinterpret_cast<filt::WarpBuf*>(smem + sizeof(sel::WarpSmem));
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + sizeof(sel::WarpSmem) +
+                                               sizeof(filt::WarpBuf));  // nb_stage
   size_t* row_off = reinterpret_cast<size_t*>(keys + nb_stage);                 // r
   float* lse = reinterpret_cast<float*>(row_off + r);                           // r
   const int b = blockIdx.x;
@@ -46,9 +50,23 @@ __global__ void __launch_bounds__(kThreads)
   __syncthreads();
   if (threadIdx.x >= 32) return;
 
-  // ---- warp 0: find_blocks on the staged row (sums in the selection
-  // kernel's order: each lane adds its blocks j = lane, lane + 32, ... in turn)
+  // ---- warp 0: find_blocks on the staged row: the threshold filter of the
+  // selection kernel first, the histogram search for a row it leaves
   const int lane = threadIdx.x;
+  const double t = tau_of(tau, bh % hq);
+  {
+    auto ld = [keys](int j) { return keys[j]; };
+    const filt::MemRow<decltype(ld)> mr{ld};
+    unsigned long long cut = 0;
+    int ncand = 0;
+    const filt::Outcome oc = filt::filter_cut(mr, nj, t, lane, FB, &cut, &ncand);
+    if (oc != filt::kUndecided) {
+      filt::emit(oc, cut, ncand, nj, NB, row, lane, FB, mask, counts, idx);
+      return;
+    }
+  }
+  // (sums in the selection kernel's order: each lane adds its blocks
+  // j = lane, lane + 32, ... in turn)
   double tot = 0.0;
   uint32_t kmax = 0;
   for (int j = lane; j < nj; j += 32) {
@@ -58,11 +76,10 @@ __global__ void __launch_bounds__(kThreads)
   }
   tot = sel::warp_sum_d(tot);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
-  const double t = static_cast<double>(tau.v[bh % hq]);
-  bool take_all;
-  uint32_t vstar;
-  int icut;
-  sel::find_cut(keys, nj, t, tot, kmax, W, lane, take_all, vstar, icut);
+  bool take_all = false;
+  uint32_t vstar = 0xFFFFFFFFu;  // selects nothing (an invalid device tau)
+  int icut = -1;
+  if (t >= 0.0) sel::find_cut(keys, nj, t, tot, kmax, W, lane, take_all, vstar, icut);
   sel::emit_row(keys, nj, NB, take_all, vstar, icut, row, lane, mask, counts, idx);
 }
 
@@ -72,7 +89,8 @@ cudaError_t launch_score_select(const Dims& D, const float* part, float* probs,
                                 const TauArg& tau, uint32_t* mask, int32_t* counts, int32_t* idx,
                                 cudaStream_t st) {
   const int nb_stage = (D.NB + 3) & ~3;
-  const size_t smem = sizeof(sel::WarpSmem) + static_cast<size_t>(nb_stage) * 4 +
+  const size_t smem = sizeof(sel::WarpSmem) + sizeof(filt::WarpBuf) +
+                      static_cast<size_t>(nb_stage) * 4 +
                       static_cast<size_t>(D.r) * (sizeof(size_t) + sizeof(float));
   cudaError_t e = cudaFuncSetAttribute(score_select_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -3,16 +3,18 @@
 // smallest set of blocks whose probability mass reaches tau), and the
 // fixed-budget Top-K / Top-Ratio selection of the pages' ablation.
 //
-// find_blocks runs as two kernels, one warp per row in each. The first walks
-// the row's ranking from per-lane top lists held in registers and adds the
-// probabilities in fp64 in ranked order, exactly as the definition does; it
-// decides almost every row of a long-context layer. The rows it cannot decide
-// go to the second, which stages the row's fp32 bit patterns (monotone in
-// value for p >= 0) in shared memory and runs the histogram search of
+// find_blocks runs as two kernels, one warp per row in each. The first is the
+// threshold filter of select_filter.cuh: it gathers the few blocks at or
+// above a threshold that already holds tau of the mass, sorts them and adds
+// their probabilities in fp64 in ranked order, exactly as the definition does;
+// it decides almost every row of a long-context layer. The rows it cannot
+// decide go to the second, which stages the row's fp32 bit patterns (monotone
+// in value for p >= 0) in shared memory and runs the histogram search of
 // select_core.cuh (shared with the fused score->select kernel). Its sums are
 // fp64 too, so its choice matches the sequential fp64 walk up to rounding in
 // the last bits.
 #include "select_core.cuh"
+#include "select_filter.cuh"
 
 namespace xattn {
 namespace {
@@ -155,148 +157,52 @@ __global__ void __launch_bounds__(kBudgetWarps * 32)
 // ---------------------------------------------------------------------------
 // find_blocks in two kernels.
 //
-// select_fast_kernel (one warp per row, no shared memory, so up to 64 rows in
-// flight per SM): while reading the row each lane keeps its kTop best blocks in
-// the find_blocks ranking (probability descending, index ascending) as 64-bit
-// rank keys in registers. Every block missing from those lists ranks at or
-// below `bound`, the best of the lanes' kTop-th entries. So taking the best
-// list head across the warp, again and again, walks the row's ranking exactly
-// for every block ranked above `bound`, and adds the probabilities in that
-// order in fp64: the same sequential sum the definition takes. If the sum
-// reaches tau above `bound`, that block is the cut. If every lane holds fewer
-// than kTop blocks, the walk covers the whole row, and a row whose sum never
-// reaches tau takes every block. Otherwise the row is marked (count -1) for
-// select_fallback_kernel, the histogram search of select_core.cuh, which runs
-// on the marked rows only. Rows with a few dominant blocks -- the long-context
-// case -- almost all finish in the fast kernel; rows whose lanes' two best
-// blocks sum to less than tau need many blocks and skip the walk.
-constexpr int kFastWarps = 8;
-constexpr int kTop = 5;
+// select_filter_kernel (one warp per row): the threshold filter of
+// select_filter.cuh. A row of at most 1024 blocks is read once into registers
+// (32 loads a lane in flight); a longer one is streamed from memory for each
+// pass (the re-reads hit L1/L2). Rows the filter cannot decide -- more than
+// filt::kCand blocks at or above the threshold that reaches tau, as in flat
+// rows -- are marked (count -1) for select_fallback_kernel, the histogram
+// search of select_core.cuh, which runs on the marked rows only.
+constexpr int kFiltWarps = 8;
 
-// Rank key of block j with fp32 bits k (sign cleared): larger ranks first.
-// ~j keeps the lower index first among equal values, and no block has key 0.
-__device__ __forceinline__ unsigned long long rank_key(uint32_t k, int j) {
-  return (static_cast<unsigned long long>(k) << 32) | static_cast<uint32_t>(~j);
-}
-
-__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long y = __shfl_xor_sync(0xffffffffu, v, o);
-    v = y > v ? y : v;
-  }
-  return v;
-}
-
-__global__ void __launch_bounds__(kFastWarps * 32)
-    select_fast_kernel(const float* __restrict__ probs, const TauArg tau, int NB, int hq,
-                       int causal, long long rows, uint32_t* __restrict__ mask,
-                       int32_t* __restrict__ counts, int32_t* __restrict__ idx) {
+__global__ void __launch_bounds__(kFiltWarps * 32, 3)
+    select_filter_kernel(const float* __restrict__ probs, const TauArg tau, int NB, int hq,
+                         int causal, long long rows, uint32_t* __restrict__ mask,
+                         int32_t* __restrict__ counts, int32_t* __restrict__ idx) {
+  __shared__ filt::WarpBuf bufs[kFiltWarps];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const long long row = static_cast<long long>(blockIdx.x) * kFastWarps + warp;
+  const long long row = static_cast<long long>(blockIdx.x) * kFiltWarps + warp;
   if (row >= rows) return;
 
   const long long bh = row / NB;
   const int b = static_cast<int>(row % NB);
   const int h = static_cast<int>(bh % hq);
   const int n = causal ? b + 1 : NB;
-  const double t = static_cast<double>(tau.v[h]);
+  const double t = tau_of(tau, h);
   const float* prow = probs + row * NB;
 
-  bool take_all = t >= 1.0;
-  unsigned long long cut = 0;  // rank key of the cut block: blocks ranked >= cut are chosen
-  if (!take_all) {
-    unsigned long long c[kTop];
+  unsigned long long cut = 0;
+  int ncand = 0;
+  filt::Outcome oc;
+  if (n <= 32 * filt::kRegU) {
+    filt::RegRow rr;
 #pragma unroll
-    for (int i = 0; i < kTop; ++i) c[i] = 0ull;
-    for (int j0 = 0; j0 < n; j0 += 8 * 32) {
-      uint32_t v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int j = j0 + u * 32 + lane;
-        v[u] = j < n ? __float_as_uint(__ldg(prow + j)) & 0x7FFFFFFFu : 0u;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int j = j0 + u * 32 + lane;
-        if (j < n) {
-          unsigned long long x = rank_key(v[u], j);
-#pragma unroll
-          for (int i = 0; i < kTop; ++i) {  // insertion into the descending list
-            const unsigned long long y = c[i];
-            c[i] = x > y ? x : y;
-            x = x > y ? y : x;
-          }
-        }
-      }
+    for (int u = 0; u < filt::kRegU; ++u) {
+      const int j = u * 32 + lane;
+      rr.k[u] = j < n ? __float_as_uint(__ldg(prow + j)) & 0x7FFFFFFFu : 0u;
     }
-    const unsigned long long bound = warp_max_u64(c[kTop - 1]);
-    // The lanes' two best entries are 64 distinct blocks, so the row's 64 best
-    // blocks hold at least their mass: if that reaches tau, the cut is among
-    // the first 64 of the walk. Otherwise the row needs many blocks (a flat
-    // row), and it goes straight to the histogram search instead of walking.
-    const double heads =
-        warp_sum_d(static_cast<double>(__uint_as_float(static_cast<uint32_t>(c[0] >> 32))) +
-                   static_cast<double>(__uint_as_float(static_cast<uint32_t>(c[1] >> 32))));
-    double acc = 0.0;
-    bool decided = false;
-    // at most kTop - 1 blocks a lane rank above bound
-    for (int it = 0; it < 32 * kTop && (heads >= t || bound == 0ull); ++it) {
-      const unsigned long long m = warp_max_u64(c[0]);
-      if (m <= bound) break;  // includes m == 0: the lists are empty
-      acc += static_cast<double>(__uint_as_float(static_cast<uint32_t>(m >> 32)));
-      if (c[0] == m) {  // the owner lane pops its head
-#pragma unroll
-        for (int i = 0; i + 1 < kTop; ++i) c[i] = c[i + 1];
-        c[kTop - 1] = 0ull;
-      }
-      if (acc >= t) {
-        cut = m;
-        decided = true;
-        break;
-      }
-    }
-    if (!decided) {
-      if (bound != 0ull) {  // the cut lies at or below bound: the histogram search decides
-        if (lane == 0) counts[row] = -1;
-        return;
-      }
-      take_all = true;  // the whole row was walked and its sum stays below tau
-    }
+    oc = filt::filter_cut(rr, n, t, lane, bufs[warp], &cut, &ncand);
+  } else {
+    auto ld = [prow](int j) { return __float_as_uint(__ldg(prow + j)) & 0x7FFFFFFFu; };
+    const filt::MemRow<decltype(ld)> mr{ld};
+    oc = filt::filter_cut(mr, n, t, lane, bufs[warp], &cut, &ncand);
   }
-
-  // emit: mask words over all NB columns, the index list in ascending order
-  const int Wn = (NB + 31) / 32;
-  uint32_t* mrow = mask + row * Wn;
-  int32_t* irow = idx + row * NB;
-  const unsigned lt = (1u << lane) - 1u;
-  int running = 0;
-  for (int j0 = 0; j0 < Wn * 32; j0 += 8 * 32) {
-    bool sel[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int j = j0 + u * 32 + lane;
-      sel[u] = false;
-      if (j < n) {
-        if (take_all) {
-          sel[u] = true;
-        } else {
-          const uint32_t k = __float_as_uint(__ldg(prow + j)) & 0x7FFFFFFFu;
-          sel[u] = rank_key(k, j) >= cut;
-        }
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int w = j0 / 32 + u;
-      if (w >= Wn) break;
-      const unsigned sb = __ballot_sync(0xffffffffu, sel[u]);
-      if (lane == 0) mrow[w] = sb;
-      if (sel[u]) irow[running + __popc(sb & lt)] = w * 32 + lane;
-      running += __popc(sb);
-    }
+  if (oc == filt::kUndecided) {
+    if (lane == 0) counts[row] = -1;
+    return;
   }
-  if (lane == 0) counts[row] = running;
+  filt::emit(oc, cut, ncand, n, NB, row, lane, bufs[warp], mask, counts, idx);
 }
 
 // The histogram search of one row (select_core.cuh), with its keys staged in
@@ -311,7 +217,7 @@ __device__ __forceinline__ void select_row_hist(const float* __restrict__ probs,
   const int b = static_cast<int>(row % NB);
   const int h = static_cast<int>(bh % hq);
   const int n = causal ? b + 1 : NB;
-  const double t = static_cast<double>(tau.v[h]);
+  const double t = tau_of(tau, h);  // valid: the fast kernel only leaves rows of valid tau
   const float* prow = probs + row * NB;
 
   double tot = 0.0;
@@ -392,8 +298,8 @@ cudaError_t launch_select_budget(const Dims& D, const float* probs, const Budget
 cudaError_t launch_select(const Dims& D, const float* probs, const TauArg& tau, uint32_t* mask,
                           int32_t* counts, int32_t* idx, int num_sms, cudaStream_t st) {
   const long long rows = static_cast<long long>(D.batch) * D.hq * D.NB;
-  const long long fast_grid = (rows + kFastWarps - 1) / kFastWarps;
-  select_fast_kernel<<<static_cast<unsigned>(fast_grid), kFastWarps * 32, 0, st>>>(
+  const long long filt_grid = (rows + kFiltWarps - 1) / kFiltWarps;
+  select_filter_kernel<<<static_cast<unsigned>(filt_grid), kFiltWarps * 32, 0, st>>>(
       probs, tau, D.NB, D.hq, D.causal, rows, mask, counts, idx);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

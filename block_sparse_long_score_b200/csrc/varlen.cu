@@ -182,8 +182,8 @@ int xattn_prefill_varlen(const void* Q, const void* K, const void* V, const xatt
     xattn_shape one = *shape;
     one.batch = 1;
     one.L = L;
-    rc = xattn_score_select(Qp + tok * qrow, Kp + tok * kvrow, &one, tau, nullptr, mask, counts,
-                            idx, score_ws, Lo.score_ws, lanes.s[lane]);
+    rc = score_select_host_tau(Qp + tok * qrow, Kp + tok * kvrow, &one, tau, nullptr, mask,
+                               counts, idx, score_ws, Lo.score_ws, lanes.s[lane]);
     if (rc == XATTN_OK)
       rc = xattn_sparse_attn(Qp + tok * qrow, Kp + tok * kvrow, Vp + tok * kvrow, &one, counts,
                              idx, Op + tok * qrow,

@@ -76,13 +76,12 @@ def _lib() -> ctypes.CDLL:
         lib.xattn_attn_workspace_bytes.restype = sz
         lib.xattn_score.argtypes = [vp, vp, sp, vp, vp, sz, vp]
         lib.xattn_score.restype = i32
-        lib.xattn_select.argtypes = [vp, ctypes.POINTER(ctypes.c_float), sp, vp, vp, vp, vp]
+        lib.xattn_select.argtypes = [vp, vp, sp, vp, vp, vp, vp]
         lib.xattn_select.restype = i32
         lib.xattn_score_pattern.argtypes = [vp, vp, sp, ctypes.POINTER(ctypes.c_int32), vp, vp,
                                             sz, vp]
         lib.xattn_score_pattern.restype = i32
-        lib.xattn_score_select.argtypes = [vp, vp, sp, ctypes.POINTER(ctypes.c_float), vp, vp,
-                                           vp, vp, vp, sz, vp]
+        lib.xattn_score_select.argtypes = [vp, vp, sp, vp, vp, vp, vp, vp, vp, sz, vp]
         lib.xattn_score_select.restype = i32
         lib.xattn_select_topk.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), sp, vp, vp, vp,
                                           vp]
@@ -279,6 +278,27 @@ def _select_outputs(probs: torch.Tensor, causal: bool, out: Optional[tuple]):
     return shape, mask, counts, idx
 
 
+def _tau_device(tau, hq: int, device) -> torch.Tensor:
+    """Per-head thresholds as the device array the C ABI reads: a CUDA float32
+    tensor of hq values is used as it is (the kernels check each value and
+    report one outside (0, 1] through xattn_get_device_status); host values
+    are checked here and copied to the device (a synchronous copy, so pass a
+    CUDA tensor inside a CUDA-graph capture)."""
+    if isinstance(tau, torch.Tensor) and tau.is_cuda:
+        _check(tau, "tau", torch.float32)
+        if tau.numel() != hq:
+            raise ValueError("tau needs one value per query head")
+        if tau.device != torch.device(device):
+            raise ValueError(f"tau must be on {device}, got {tau.device}")
+        return tau
+    vals = [float(v) for v in (tau.tolist() if hasattr(tau, "tolist") else tau)]
+    if len(vals) != hq:
+        raise ValueError("tau needs one value per query head")
+    if not all(0.0 < v <= 1.0 for v in vals):
+        raise ValueError("every tau must lie in (0, 1]")
+    return torch.tensor(vals, dtype=torch.float32).to(device)
+
+
 def _per_head(values, hq: int, name: str, kind):
     vals = [kind(v) for v in values]
     if len(vals) != hq:
@@ -286,25 +306,27 @@ def _per_head(values, hq: int, name: str, kind):
     return vals
 
 
-def xattn_select(probs: torch.Tensor, tau: Sequence[float], causal: bool,
-                 out: Optional[tuple] = None):
-    """find_blocks on every row of P. Returns (mask uint32 [.., NB, ceil(NB/32)] as
-    int32, counts int32 [.., NB], idx int32 [.., NB, NB])."""
+def xattn_select(probs: torch.Tensor, tau, causal: bool, out: Optional[tuple] = None):
+    """find_blocks on every row of P with per-head thresholds ``tau`` (a CUDA
+    float32 tensor [hq], read on the device, or host values). Returns (mask
+    uint32 [.., NB, ceil(NB/32)] as int32, counts int32 [.., NB], idx int32
+    [.., NB, NB])."""
     shape, mask, counts, idx = _select_outputs(probs, causal, out)
-    taus = _per_head(tau, shape.hq, "tau", float)
-    tarr = (ctypes.c_float * shape.hq)(*taus)
     with torch.cuda.device(probs.device):
-        rc = _lib().xattn_select(probs.data_ptr(), tarr, ctypes.byref(shape), mask.data_ptr(),
-                                 counts.data_ptr(), idx.data_ptr(), _stream(probs.device))
+        tdev = _tau_device(tau, shape.hq, probs.device)
+        rc = _lib().xattn_select(probs.data_ptr(), tdev.data_ptr(), ctypes.byref(shape),
+                                 mask.data_ptr(), counts.data_ptr(), idx.data_ptr(),
+                                 _stream(probs.device))
     _raise("xattn_select", rc)
     return mask, counts, idx
 
 
 def xattn_score_select(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal: bool,
-                       tau: Sequence[float], probs: Optional[torch.Tensor] | bool = None,
+                       tau, probs: Optional[torch.Tensor] | bool = None,
                        out: Optional[tuple] = None, workspace: Optional[torch.Tensor] = None):
-    """Scoring and find_blocks in one call (P stays on chip). Returns (mask,
-    counts, idx), or (probs, mask, counts, idx) when probs is True or a tensor."""
+    """Scoring and find_blocks in one call (P stays on chip); ``tau`` as for
+    xattn_select. Returns (mask, counts, idx), or (probs, mask, counts, idx)
+    when probs is True or a tensor."""
     _check(Q, "Q")
     _check(K, "K", Q.dtype)
     shape = _shape_of(Q, K, B, S, causal)
@@ -323,17 +345,17 @@ def xattn_score_select(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal:
     else:
         mask, counts, idx = out
     _check_select_outputs(mask, counts, idx, shape.batch, shape.hq, NB)
-    taus = _per_head(tau, shape.hq, "tau", float)
-    tarr = (ctypes.c_float * shape.hq)(*taus)
     need = xattn_score_workspace_bytes(shape)
     if workspace is None:
         workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
     _check(workspace, "workspace")
     _same_device(Q, K, probs if want_p else None, mask, counts, idx, workspace)
     with torch.cuda.device(Q.device):
-            rc = _lib().xattn_score_select(Q.data_ptr(), K.data_ptr(), ctypes.byref(shape), tarr,
-                                       probs.data_ptr() if want_p else None, mask.data_ptr(),
-                                       counts.data_ptr(), idx.data_ptr(), workspace.data_ptr(),
+        tdev = _tau_device(tau, shape.hq, Q.device)
+        rc = _lib().xattn_score_select(Q.data_ptr(), K.data_ptr(), ctypes.byref(shape),
+                                       tdev.data_ptr(), probs.data_ptr() if want_p else None,
+                                       mask.data_ptr(), counts.data_ptr(), idx.data_ptr(),
+                                       workspace.data_ptr(),
                                        workspace.numel() * workspace.element_size(),
                                        _stream(Q.device))
     _raise("xattn_score_select", rc)

@@ -32,8 +32,9 @@
  * - Arguments are checked on the host before anything is launched. A failed
  *   check returns a negative xattn_status and launches nothing.
  * - Device-side faults that a kernel can detect on its own (a pipeline wait
- *   that exceeded its time limit) are recorded in a per-device status word
- *   that xattn_get_device_status reads and clears. Kernels never trap.
+ *   that exceeded its time limit, a device-resident tau out of range) are
+ *   recorded in a per-device status word that xattn_get_device_status reads
+ *   and clears. Kernels never trap.
  *
  * Two further calls run the pages' ablation variants through the same
  * kernels: xattn_score_pattern (diagonal / random sampling instead of the
@@ -122,13 +123,19 @@ int xattn_score(const void* Q, const void* K, const xattn_shape* shape, float* p
  * Sums are accumulated in fp64.
  *
  * probs: fp32 [batch, hq, NB, NB], device.
- * tau:   HOST pointer to hq floats, each in (0, 1]; INVALID_ARG otherwise.
+ * tau:   DEVICE pointer to hq floats (per-head thresholds, read by the kernels
+ *        when they run, so a captured CUDA graph picks up new values written
+ *        there). Each must lie in (0, 1]. A value outside (or NaN) cannot be
+ *        seen on the host: the kernels select nothing in that head's rows
+ *        (counts 0, mask words 0) and record the fault, which the next
+ *        xattn_get_device_status returns as XATTN_ERR_INVALID_ARG.
  * mask:   out, uint32 [batch, hq, NB, ceil(NB/32)]; bit (j % 32) of word j / 32
  *         is set iff block j is selected. Fully written.
  * counts: out, int32 [batch, hq, NB], the number of selected blocks.
  * idx:    out, int32 [batch, hq, NB, NB]; the first counts[...] entries of a
  *         row are the selected block indices in ascending order. The rest of
  *         the row is left unwritten.
+ * Errors (returned): INVALID_ARG (NULL pointer, bad shape), UNSUPPORTED, CUDA.
  */
 int xattn_select(const float* probs, const float* tau, const xattn_shape* shape,
                  uint32_t* mask, int32_t* counts, int32_t* idx, void* stream);
@@ -139,7 +146,8 @@ int xattn_select(const float* probs, const float* tau, const xattn_shape* shape,
  * find_blocks on it straight from on-chip memory, so P makes no round trip
  * through HBM (§2.2: block scores, then the threshold selection).
  *
- * tau:   HOST pointer to hq floats in (0, 1], as for xattn_select.
+ * tau:   DEVICE pointer to hq floats in (0, 1], read and checked by the
+ *        kernels as for xattn_select.
  * probs: out, optional (may be NULL): fp32 [batch, hq, NB, NB], bit-identical
  *        to xattn_score's output when given.
  * mask, counts, idx: out, as for xattn_select, and bit-identical to
@@ -296,7 +304,9 @@ size_t xattn_prefill_host_workspace_bytes(const xattn_shape* shape, int kv_heads
  *          memory (page-locked, e.g. from cudaHostAlloc, for the copies to
  *          overlap; pageable memory gives the same results more slowly) or
  *          device memory. Not modified.
- * tau:     HOST pointer to hq floats in (0, 1], as for xattn_select.
+ * tau:     HOST pointer to hq floats in (0, 1], checked before anything is
+ *          launched (INVALID_ARG) and passed to the kernels by value: this
+ *          host-facing call takes its thresholds from the host.
  * O:       out, [batch, hq, L, d] of the same type, host or device memory.
  * lse:     out, optional (may be NULL), fp32 [batch, hq, L], as for
  *          xattn_sparse_attn.
@@ -340,7 +350,8 @@ size_t xattn_prefill_varlen_workspace_bytes(const xattn_shape* shape, int nseq,
  * fp32 arrays at T_i * hq. All DEVICE pointers, 16-byte aligned for bf16.
  * shape: hq, hkv, d, B, S, causal and dtype apply to every sequence; its
  * batch and L are ignored.
- * tau: HOST pointer to hq floats in (0, 1].
+ * tau: HOST pointer to hq floats in (0, 1], checked before anything is
+ *      launched and passed to the kernels by value.
  * ws / ws_bytes: DEVICE workspace of at least
  *          xattn_prefill_varlen_workspace_bytes(shape, nseq, seqlens) bytes,
  *          256-byte aligned.
@@ -363,7 +374,9 @@ int xattn_prefill_varlen(const void* Q, const void* K, const void* V, const xatt
 /*
  * Synchronises `stream`, then reads and clears the current device's status
  * word. Returns XATTN_OK, XATTN_ERR_TIMEOUT if a kernel gave up a bounded
- * wait since the last call, or XATTN_ERR_CUDA if the stream reports an error.
+ * wait since the last call, XATTN_ERR_INVALID_ARG if a selection kernel met a
+ * device-resident tau outside (0, 1], or XATTN_ERR_CUDA if the stream reports
+ * an error. When several faults happened, the last one recorded is returned.
  */
 int xattn_get_device_status(void* stream);
 

@@ -100,7 +100,12 @@ int main(int argc, char** argv) {
 
   cudaStream_t st;
   CHECK_CUDA(cudaStreamCreate(&st));
-  CHECK_XATTN(xattn_score_select(Q, K, &sh, tau, NULL, mask, counts, idx, ws_s, ws_s_bytes, st));
+  /* per-head thresholds live in device memory (the kernels read them there) */
+  float* tau_d;
+  CHECK_CUDA(cudaMalloc((void**)&tau_d, sizeof(float) * sh.hq));
+  CHECK_CUDA(cudaMemcpy(tau_d, tau, sizeof(float) * sh.hq, cudaMemcpyHostToDevice));
+  CHECK_XATTN(xattn_score_select(Q, K, &sh, tau_d, NULL, mask, counts, idx, ws_s, ws_s_bytes,
+                                 st));
   CHECK_XATTN(xattn_sparse_attn(Q, K, V, &sh, counts, idx, O, NULL, ws_a, ws_a_bytes, st));
   CHECK_XATTN(xattn_get_device_status(st));
 
@@ -109,7 +114,7 @@ int main(int argc, char** argv) {
   if (!f || fwrite(host, 2, nq, f) != nq) return 8;
   fclose(f);
   cudaFree(Q); cudaFree(K); cudaFree(V); cudaFree(O); cudaFree(ws_s); cudaFree(ws_a);
-  cudaFree(mask); cudaFree(counts); cudaFree(idx);
+  cudaFree(mask); cudaFree(counts); cudaFree(idx); cudaFree(tau_d);
   cudaStreamDestroy(st);
   free(host);
   free(tau);

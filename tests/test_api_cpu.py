@@ -76,9 +76,23 @@ def test_null_pointers_and_workspace(lib):
 
 @pytest.mark.parametrize("tau", [0.0, -0.5, 1.5, float("nan")])
 def test_tau_out_of_range(lib, tau):
+    """The whole-step calls take tau in host memory and check it before any
+    launch. (xattn_select and xattn_score_select read tau from device memory;
+    the kernels check it there, which the GPU tests cover.)"""
     s = X.make_shape(1, 2, 2, 1024, 128, 128, 8, True, "bf16")
     t = (ctypes.c_float * 2)(0.9, tau)
-    assert lib.xattn_select(FAKE, t, ctypes.byref(s), FAKE, FAKE, FAKE, None) == -1
+    assert lib.xattn_prefill_host(FAKE, FAKE, FAKE, ctypes.byref(s), t, FAKE, None, 0, FAKE,
+                                  1 << 40, None) == -1
+    lens = (ctypes.c_int32 * 1)(1024)
+    assert lib.xattn_prefill_varlen(FAKE, FAKE, FAKE, ctypes.byref(s), 1, lens, t, FAKE, None,
+                                    FAKE, 1 << 40, None) == -1
+
+
+def test_null_tau_refused(lib):
+    s = X.make_shape(1, 2, 2, 1024, 128, 128, 8, True, "bf16")
+    assert lib.xattn_select(FAKE, None, ctypes.byref(s), FAKE, FAKE, FAKE, None) == -1
+    assert lib.xattn_score_select(FAKE, FAKE, ctypes.byref(s), None, None, FAKE, FAKE, FAKE,
+                                  FAKE, 1 << 40, None) == -1
 
 
 def test_misaligned_bf16_pointer(lib):
@@ -136,10 +150,8 @@ def test_budget_null_pointers(lib):
 
 def test_score_select_host_checks(lib):
     s = X.make_shape(1, 2, 2, 1024, 128, 128, 8, True, "bf16")
-    good = (ctypes.c_float * 2)(0.9, 0.9)
-    bad = (ctypes.c_float * 2)(0.9, 1.5)
+    good = FAKE   # tau is a device pointer here: its values are checked by the kernels
     f = lib.xattn_score_select
-    assert f(FAKE, FAKE, ctypes.byref(s), bad, None, FAKE, FAKE, FAKE, FAKE, 1 << 40, None) == -1
     assert f(FAKE, FAKE, ctypes.byref(s), None, None, FAKE, FAKE, FAKE, FAKE, 1 << 40, None) == -1
     assert f(FAKE, FAKE, ctypes.byref(s), good, None, None, FAKE, FAKE, FAKE, 1 << 40, None) == -1
     assert f(None, FAKE, ctypes.byref(s), good, None, FAKE, FAKE, FAKE, FAKE, 1 << 40, None) == -1

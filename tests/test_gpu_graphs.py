@@ -22,7 +22,7 @@ DEV = "cuda:0"
 
 def _step(Q, K, V, prob, out):
     P = xattn_score(Q, K, prob.B, prob.S, prob.causal, probs=out["P"], workspace=out["ws_s"])
-    xattn_select(P, prob.tau.tolist(), prob.causal, out=(out["mask"], out["counts"], out["idx"]))
+    xattn_select(P, out["tau"], prob.causal, out=(out["mask"], out["counts"], out["idx"]))
     xattn_sparse_attn(Q, K, V, out["counts"], out["idx"], prob.B, prob.causal, out=out["O"],
                       lse=out["lse"], workspace=out["ws_a"])
 
@@ -43,6 +43,7 @@ def _buffers(prob, Q):
         "lse": torch.empty(Q.shape[:3], device=DEV),
         "ws_s": torch.empty(xattn_score_workspace_bytes(shape), device=DEV, dtype=torch.uint8),
         "ws_a": torch.empty(xattn_attn_workspace_bytes(shape), device=DEV, dtype=torch.uint8),
+        "tau": torch.tensor(prob.tau.tolist(), dtype=torch.float32, device=DEV),
     }
 
 
@@ -100,12 +101,13 @@ def test_fused_call_and_varlen_replay_in_a_graph():
 
     p = probs[2]
     Qd, Kd = p.Q.to(DEV), p.K.to(DEV)
-    m1, c1, i1 = xattn_score_select(Qd, Kd, p.B, p.S, p.causal, tau)
+    tau_d = torch.tensor(tau, dtype=torch.float32, device=DEV)
+    m1, c1, i1 = xattn_score_select(Qd, Kd, p.B, p.S, p.causal, tau_d)
     torch.cuda.synchronize()
     outs = (torch.zeros_like(m1), torch.zeros_like(c1), torch.zeros_like(i1))
     g2 = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g2):
-        xattn_score_select(Qd, Kd, p.B, p.S, p.causal, tau, out=outs)
+        xattn_score_select(Qd, Kd, p.B, p.S, p.causal, tau_d, out=outs)
     g2.replay()
     torch.cuda.synchronize()
     assert torch.equal(outs[0], m1) and torch.equal(outs[1], c1)
@@ -132,3 +134,56 @@ def test_host_buffer_call_replays_in_a_graph():
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(Oh, eager)
+
+
+def test_replayed_step_reads_new_tau_from_the_device():
+    """Per-head tau lives in a device array the kernels read at run time, so a
+    captured step takes new thresholds written into that array, without
+    capturing again. Every head's tau changes between the replays."""
+    p = make_problem("c1", L=4096, hq=4, hkv=2, seed=50)
+    Q, K, V = p.Q.to(DEV), p.K.to(DEV), p.V.to(DEV)
+    buf = _buffers(p, Q)
+    _step(Q, K, V, p, buf)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        _step(Q, K, V, p, buf)
+    for taus in ([0.5, 0.6, 0.7, 0.8], [0.99, 0.95, 0.9, 1.0]):
+        buf["tau"].copy_(torch.tensor(taus, dtype=torch.float32))
+        g.replay()
+        torch.cuda.synchronize()
+        assert xattn_get_device_status() == 0
+        ref = _buffers(p, Q)
+        ref["tau"].copy_(torch.tensor(taus, dtype=torch.float32))
+        _step(Q, K, V, p, ref)
+        torch.cuda.synchronize()
+        for k in ("mask", "counts", "O"):
+            assert torch.equal(buf[k], ref[k]), (taus, k)
+    # tau = 1 on the last head selects every causally allowed block
+    NB = p.NB
+    assert torch.equal(buf["counts"][0, 3].cpu(), torch.arange(1, NB + 1, dtype=torch.int32))
+
+
+@pytest.mark.parametrize("bad", [0.0, -0.5, 1.5, float("nan")])
+def test_invalid_device_tau_is_reported(bad):
+    """A device-resident tau outside (0, 1] cannot be checked on the host: the
+    kernels check it, select nothing for that head and report INVALID_ARG
+    through the device status, for both selection calls; the other heads are
+    unaffected and the context stays usable."""
+    p = make_problem("c1", L=2048, hq=2, hkv=1, seed=51)
+    Q, K = p.Q.to(DEV), p.K.to(DEV)
+    assert xattn_get_device_status() == 0
+    tau_ok = torch.tensor([0.9, 0.9], dtype=torch.float32, device=DEV)
+    tau_bad = torch.tensor([0.9, bad], dtype=torch.float32, device=DEV)
+    P = xattn_score(Q, K, p.B, p.S, p.causal)
+    m_ok, c_ok, i_ok = xattn_select(P, tau_ok, p.causal)
+    torch.cuda.synchronize()
+    assert xattn_get_device_status() == 0
+    for call in (lambda: xattn_select(P, tau_bad, p.causal),
+                 lambda: xattn_score_select(Q, K, p.B, p.S, p.causal, tau_bad)):
+        m, c, _ = call()
+        torch.cuda.synchronize()
+        assert xattn_get_device_status() == -1          # XATTN_ERR_INVALID_ARG
+        assert xattn_get_device_status() == 0           # read and cleared
+        assert torch.equal(c[0, 0], c_ok[0, 0]) and torch.equal(m[0, 0], m_ok[0, 0])
+        assert int(c[0, 1].abs().sum()) == 0 and int(m[0, 1].abs().sum()) == 0

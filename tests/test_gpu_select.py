@@ -99,3 +99,26 @@ def test_many_equal_values_at_the_cut():
             P[0, h, b, 200:] = 1.0 / 8192
             P[0, h, b, 7] = 0.25
     _check(P, [0.3, 0.45], False)
+
+
+def test_cut_below_the_first_thresholds_and_zero_rows():
+    """Rows whose cut lies 9 and 15 octaves below the maximum (the filter's
+    first thresholds hold too little mass, so lower ones are tried), rows with
+    more candidates than the filter sorts (left to the histogram search), and
+    all-zero rows (the sum never reaches tau: every allowed block)."""
+    NB = 700
+    rng = np.random.default_rng(5)
+    P = np.zeros((1, 4, NB, NB))
+    for h in range(4):
+        for b in range(NB):
+            n = b + 1
+            row = np.full(n, 1e-9)
+            row[rng.integers(0, n)] = 0.5
+            k = min(n, [20, 20, 200, 0][h])
+            if k:
+                pos = rng.choice(n, size=k, replace=False)
+                row[pos] = 0.5 * 2.0 ** -(9 if h == 0 else (15 if h == 1 else 10))
+            if h == 3 and b % 3 == 0:
+                row[:] = 0.0
+            P[0, h, b, :n] = row
+    _check(P, [0.5 + 0.5 * 2.0 ** -9 * 7.5, 0.5 + 0.5 * 2.0 ** -15 * 12.5, 0.6, 0.9], True)

@@ -3,6 +3,7 @@ the max-over-ranks timing reduction. The path itself has no collective."""
 import os
 import socket
 
+import numpy as np
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
@@ -53,3 +54,21 @@ def test_single_process_is_identity():
     import bench
     assert bench.max_over_ranks(3.25) == 3.25
     assert bench.whole_job_ms_per_layer(8.0, 1) == 8.0
+
+
+def test_head_split_host_logic():
+    """--split heads: each rank keeps its KV-head range of the same layer (with
+    the query heads and thresholds of those heads), and a layer takes the
+    slowest rank's step instead of being one of `world` replicas."""
+    import bench
+    from block_sparse_long_score_b200.synth import make_problem
+    prob = make_problem("c1", L=1024, hq=8, hkv=4)
+    parts = [bench.local_heads(prob, r, 3) for r in range(3)]
+    assert [(p.hq, p.hkv) for p in parts] == [(4, 2), (2, 1), (2, 1)]
+    assert torch.equal(torch.cat([p.Q for p in parts], dim=1), prob.Q)
+    assert torch.equal(torch.cat([p.K for p in parts], dim=1), prob.K)
+    assert torch.equal(torch.cat([p.V for p in parts], dim=1), prob.V)
+    assert list(np.concatenate([p.tau for p in parts])) == list(prob.tau)
+    assert all(p.Q.is_contiguous() and p.K.is_contiguous() for p in parts)
+    assert bench.whole_job_ms_per_layer(12.0, 4, "heads") == 12.0
+    assert bench.whole_job_ms_per_layer(12.0, 4, "replicas") == 3.0
