@@ -3,12 +3,16 @@
 
 One step = one layer's prefill attention on the 128K Llama-3.1-8B-shaped
 workload (32 query / 8 KV heads, d = 128, L = 131072, bf16, causal, B = 128,
-S = 16, per-head tau from {0.8, 0.85, 0.9, 0.95}): xattn_score, xattn_select
-and xattn_sparse_attn through the C ABI, inputs resident in HBM.
+S = 16, per-head tau from {0.8, 0.85, 0.9, 0.95}) through the package's
+one-call API, prefill_attention (xattn_score_select, then xattn_sparse_attn,
+through the C ABI), inputs resident in HBM. The per-call split (and the
+three-call path that writes P, for the selection kernel's own figures) is
+timed in separate loops outside the headline's timed region.
 
 Prints one JSON line (rank 0). Multi-GPU runs (torchrun) are independent
-replicas: every rank runs the same layer, with no collective in the data path;
-the timed region is bracketed by a barrier and the max over ranks is reported.
+replicas by default: every rank runs the same layer, with no collective in
+the data path; --split heads cuts one layer into KV-head ranges instead. The
+timed region is bracketed by a barrier and the max over ranks is reported.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
@@ -337,6 +341,7 @@ def problem_overrides(args) -> dict:
 def run_ours(args, rank: int, world: int, local: int) -> None:
     from block_sparse_long_score_b200 import (xattn_score, xattn_select, xattn_sparse_attn,
                                               xattn_score_select, xattn_get_device_status,
+                                              prefill_attention,
                                               xattn_score_workspace_bytes,
                                               xattn_attn_workspace_bytes, make_shape,
                                               xattn_prefill_host,
@@ -365,39 +370,67 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     tau_d = torch.tensor(taus, dtype=torch.float32, device=dev)   # per-head tau, device-resident
     stream = torch.cuda.current_stream(dev)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-
-    def step(ev=None):
-        if ev:
-            ev[0].record(stream)
-        if args.fused:
-            # scoring, block sums and find_blocks in one call (P stays on chip);
-            # its time is reported under "score", "select" is 0
-            xattn_score_select(Q, K, prob.B, prob.S, prob.causal, tau_d,
-                               out=(mask, counts, idx), workspace=ws_s)
-            if ev:
-                ev[1].record(stream)
-        else:
-            xattn_score(Q, K, prob.B, prob.S, prob.causal, probs=probs, workspace=ws_s)
-            if ev:
-                ev[1].record(stream)
-            xattn_select(probs, tau_d, prob.causal, out=(mask, counts, idx))
-        if ev:
-            ev[2].record(stream)
-        xattn_sparse_attn(Q, K, V, counts, idx, prob.B, prob.causal, out=out, workspace=ws_a)
-        if gather:
-            # the whole layer's O on every rank (NCCL all-gather of the head ranges)
-            from block_sparse_long_score_b200.shard import gather_heads
-            gather_heads(out, layer_hq, layer_hkv)
-        if ev:
-            ev[3].record(stream)
-
+    bufs = {"mask": mask, "counts": counts, "idx": idx, "out": out, "ws_score": ws_s,
+            "ws_attn": ws_a}
     gather = args.split == "heads" and args.gather and world > 1
+
+    def gather_o():
+        # the whole layer's O on every rank (NCCL all-gather of the head ranges)
+        from block_sparse_long_score_b200.shard import gather_heads
+        gather_heads(out, layer_hq, layer_hkv)
+
+    def step():
+        """One step through the product's API: prefill_attention (scoring fused
+        with the block sums and find_blocks, then the sparse attention), or the
+        three separate calls with --two-call."""
+        if args.two_call:
+            xattn_score(Q, K, prob.B, prob.S, prob.causal, probs=probs, workspace=ws_s)
+            xattn_select(probs, tau_d, prob.causal, out=(mask, counts, idx))
+            xattn_sparse_attn(Q, K, V, counts, idx, prob.B, prob.causal, out=out,
+                              workspace=ws_a)
+        else:
+            prefill_attention(Q, K, V, prob.B, prob.S, tau_d, prob.causal, buffers=bufs)
+        if gather:
+            gather_o()
+
+    def split_fused(ev):
+        """The product path's two calls with events between them."""
+        ev[0].record(stream)
+        xattn_score_select(Q, K, prob.B, prob.S, prob.causal, tau_d,
+                           out=(mask, counts, idx), workspace=ws_s)
+        ev[1].record(stream)
+        xattn_sparse_attn(Q, K, V, counts, idx, prob.B, prob.causal, out=out, workspace=ws_a)
+        ev[2].record(stream)
+
+    def split_two(ev):
+        """The three-call path (P written to HBM, then find_blocks on it) with
+        events between the calls: the per-kernel figures of scoring and
+        selection."""
+        ev[0].record(stream)
+        xattn_score(Q, K, prob.B, prob.S, prob.causal, probs=probs, workspace=ws_s)
+        ev[1].record(stream)
+        xattn_select(probs, tau_d, prob.causal, out=(mask, counts, idx))
+        ev[2].record(stream)
+        xattn_sparse_attn(Q, K, V, counts, idx, prob.B, prob.causal, out=out, workspace=ws_a)
+        ev[3].record(stream)
+
+    def timed_split(fn, nev):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)]
+               for _ in range(args.steps)]
+        for _ in range(2):
+            fn(evs[0])
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            fn(evs[i])
+        torch.cuda.synchronize(dev)
+        return [max_over_ranks(sum(e[k].elapsed_time(e[k + 1]) for e in evs) / args.steps, dev)
+                for k in range(nev - 1)]
+
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
     if xattn_get_device_status(dev) != 0:
-        raise RuntimeError("device status reports a kernel time-out")
+        raise RuntimeError("device status reports a kernel fault")
     selected = int(counts.sum().item())
     allowed = prob.batch * prob.hq * (NB * (NB + 1) // 2 if prob.causal else NB * NB)
     density = selected / allowed
@@ -410,22 +443,24 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     clocks.start()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    per = {"score": 0.0, "select": 0.0, "sparse_attn": 0.0}
     t_start.record(stream)
     for i in range(args.steps):
-        step(evs[i])
+        step()
     t_end.record(stream)
     torch.cuda.synchronize(dev)
-    for ev in evs:
-        per["score"] += ev[0].elapsed_time(ev[1])
-        per["select"] += ev[1].elapsed_time(ev[2])
-        per["sparse_attn"] += ev[2].elapsed_time(ev[3])
     if dist:
         torch.distributed.barrier()
     clk = clocks.stop()
     total_ms = t_start.elapsed_time(t_end)
     ms_step = max_over_ranks(total_ms / args.steps, dev)
-    per = {k: v / args.steps for k, v in per.items()}
+
+    # per-call split, outside the headline's timed region
+    t_ss, t_attn = timed_split(split_fused, 3)
+    t_sc, t_sel, t_attn2 = timed_split(split_two, 4)
+    per = {"score_select": t_ss, "sparse_attn": t_attn}
+    per_two = {"score": t_sc, "select": t_sel, "sparse_attn": t_attn2}
+    if xattn_get_device_status(dev) != 0:
+        raise RuntimeError("device status reports a kernel fault")
 
     # end to end through the public API, every step: Q, K, V from pinned host
     # memory, the whole step, O back to pinned host memory. xattn_prefill_host
@@ -492,8 +527,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     # attention the block-sparse step replaces, for context
     dense_ms = None
     if not args.no_dense:
-        if args.fused:
-            probs.zero_()   # the fused path never wrote P; tau = 1 selects all either way
+        # P from the three-call split above; tau = 1 selects every allowed block
         xattn_select(probs, torch.ones_like(tau_d), prob.causal, out=(mask, counts, idx))
         xattn_sparse_attn(Q, K, V, counts, idx, prob.B, prob.causal, out=out, workspace=ws_a)
         torch.cuda.synchronize(dev)
@@ -516,22 +550,27 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     attn_tflops = attn_flops / (per["sparse_attn"] * 1e-3) / 1e12
     pairs = prob.hq * prob.batch * (NB * (NB + 1) // 2 if prob.causal else NB * NB)
     score_flops = 2.0 * prob.B * prob.B * prob.d / prob.S * pairs
-    score_tflops = score_flops / (per["score"] * 1e-3) / 1e12
+    ss_tflops = score_flops / (per["score_select"] * 1e-3) / 1e12
+    score_tflops = score_flops / (per_two["score"] * 1e-3) / 1e12
+    # selection's algorithmic bytes: the causal half of P read (4 B per allowed
+    # block), the lists written (4 B per selected block), mask words and counts
     sel_bytes = 4.0 * pairs + 4.0 * selected + 4.0 * W * NB * prob.hq * prob.batch + \
         4.0 * NB * prob.hq * prob.batch
-    sel_gbs = sel_bytes / (per["select"] * 1e-3) / 1e9 if not args.fused else None
+    sel_gbs = sel_bytes / (per_two["select"] * 1e-3) / 1e9
     dense = dense_equiv_flops(prob)
     dense_tflops = dense / (ms_step * 1e-3) / 1e12
     peak_attn, peak_source = bf16_peak_for_clocks(pk, clk)
-    # the roofline object describes the call with the largest share of the step
-    if per["score"] >= per["sparse_attn"]:
-        dom, dom_tflops = "score", score_tflops
-        dom_kernel = ("xattn_score_select (score_tc_kernel + score_select_kernel)" if args.fused
-                      else "xattn_score (score_tc_kernel + score_reduce_kernel)")
+    # the roofline object describes the call with the largest share of the
+    # headline step (the product path)
+    if per["score_select"] >= per["sparse_attn"]:
+        dom, dom_tflops = "score_select", ss_tflops
+        dom_kernel = "xattn_score_select (score_tc_kernel + score_select_kernel)"
     else:
         dom, dom_tflops = "sparse_attn", attn_tflops
         dom_kernel = "xattn_sparse_attn (sched_kernel + attn_tc_kernel)"
-    traffic = None if (args.heads or args.fused) else TRAFFIC_BYTES.get((args.config, dom))
+    traffic = None if args.heads else TRAFFIC_BYTES.get((args.config, dom))
+    path = ("xattn_score + xattn_select + xattn_sparse_attn" if args.two_call
+            else "prefill_attention (xattn_score_select + xattn_sparse_attn)")
     line = {
         "metric": METRIC,
         "value": whole_job_ms_per_layer(ms_step, world, args.split),
@@ -546,13 +585,13 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
         "dtype": "bf16",
         "data": "synthetic (seeded Llama-3.1-8B-shaped Q/K/V with planted sinks and slash bands)",
         "config": dict(workload_config(prob), **split_config(args, world, layer_hq, layer_hkv),
-                       path="xattn_score_select + xattn_sparse_attn" if args.fused
-                       else "xattn_score + xattn_select + xattn_sparse_attn"),
+                       path=path),
         "dense_equiv_tflops": dense_tflops,
         "pct_peak": 100.0 * dense_tflops / pk["bf16"],
         "density": density,
         "per_kernel_ms": per,
-        "score_select_share": (per["score"] + per["select"]) / ms_step,
+        "per_kernel_ms_three_calls": per_two,
+        "score_select_share": per["score_select"] / ms_step,
         "graph_replay_ms_per_step": graph_ms,
         "dense_mask_attn": None if dense_ms is None else {
             "ms": dense_ms,
@@ -562,8 +601,9 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
             "note": "xattn_sparse_attn on the tau = 1 mask (every allowed block)",
         },
         "kernel_fracs": {
+            "score_select": {"tflops": ss_tflops, "frac": ss_tflops / peak_attn},
             "score": {"tflops": score_tflops, "frac": score_tflops / peak_attn},
-            "select": {"gbs": sel_gbs, "frac": sel_gbs / pk["hbm_gbs"] if sel_gbs else None},
+            "select": {"gbs": sel_gbs, "frac": sel_gbs / pk["hbm_gbs"]},
             "sparse_attn": {"tflops": attn_tflops, "frac": attn_tflops / peak_attn},
         },
         "roofline": {
@@ -587,7 +627,10 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
         # the same copies and calls one after another on one stream, for context
         "e2e_serial": {"value": whole_job_ms_per_layer(e2e_serial_ms, world, args.split),
                        "unit": "ms/layer"},
-        "gpu_launches": (4 if args.fused else 6) * args.steps,
+        # library kernels launched in the headline's timed region: score_tc +
+        # score_select + sched + attn_tc a step (three calls: score_tc +
+        # score_reduce + select_filter + select_fallback + sched + attn_tc)
+        "gpu_launches": (6 if args.two_call else 4) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -661,8 +704,9 @@ def main() -> None:
     ap.add_argument("--config", default=WORKLOAD, choices=["c1", "c2", "c3", "c4"],
                     help="workload (default c2, the 128K layer the metric is quoted on)")
     ap.add_argument("--stride", type=int, default=0, help="stride S for the video layer (c4)")
-    ap.add_argument("--fused", action="store_true",
-                    help="run scoring and selection as one call (xattn_score_select)")
+    ap.add_argument("--two-call", action="store_true",
+                    help="time the three separate calls (P written to HBM) instead of the "
+                         "product path prefill_attention")
     ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
                     help="multi-GPU: whole-layer replicas (default) or one layer cut into "
                          "contiguous KV-head ranges, one per rank")

@@ -21,4 +21,4 @@ from .xattn import (  # noqa: F401
     xattn_prefill_host_workspace_bytes, xattn_prefill_varlen,
     xattn_prefill_varlen_workspace_bytes, xattn_check_lists,
 )
-from .pipeline import prefill_attention  # noqa: F401
+from .pipeline import prefill_attention, prefill_buffers  # noqa: F401

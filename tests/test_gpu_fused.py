@@ -50,6 +50,8 @@ def _assert_same_lists(c1, i1, c2, i2):
     ("c2", dict(L=8192, hq=4, hkv=1)),
     ("c4", dict(frames=3, frame_tokens=640, hq=2, S=16)),
     ("c4", dict(frames=3, frame_tokens=640, hq=2, S=4)),
+    ("c1", dict(L=76800, hq=2, hkv=1)),          # rows of 513..600 blocks: two passes (r = 16)
+    ("c4", dict(frames=3, frame_tokens=12800, hq=1, S=4)),  # 300-block rows, r = 32
 ])
 def test_fused_equals_two_calls(name, kw):
     prob = make_problem(name, **kw)
@@ -95,3 +97,27 @@ def test_fused_full_size():
     assert torch.equal(P, P2)
     assert torch.equal(m1, m2) and torch.equal(m1, m3)
     _assert_same_lists(c1, i1, c2, i2)
+
+
+@pytest.mark.parametrize("name,kw,blocks", [
+    ("c4", dict(frames=3, frame_tokens=12800, hq=1, S=4), [0, 150, 299]),
+    ("c1", dict(L=76800, hq=1, hkv=1), [0, 511, 512, 599]),
+])
+def test_long_rows_match_oracle(name, kw, blocks):
+    """Rows longer than one register pass of the reduction (two passes over the
+    partials) against the oracle's P, and its find_blocks on the GPU's P."""
+    prob = make_problem(name, **kw)
+    Q, K = prob.Q.to(DEV), prob.K.to(DEV)
+    P, mask, counts, idx = xattn_score_select(Q, K, prob.B, prob.S, prob.causal,
+                                              prob.tau.tolist(), probs=True)
+    torch.cuda.synchronize()
+    Pg = PT.to_np(P).astype(np.float64)
+    Pref = O.block_probs(prob.Q, prob.K, prob.B, prob.S, prob.causal, heads=[0],
+                         q_blocks=blocks)
+    assert PT.check_probs(Pg[0, 0, blocks], Pref[0, 0, blocks]) <= 1.0
+    mb = PT.mask_to_bool(PT.to_np(mask), prob.NB)
+    for b in blocks:
+        n = b + 1 if prob.causal else prob.NB
+        want = np.zeros(prob.NB, bool)
+        want[O.find_blocks(Pg[0, 0, b, :n], float(prob.tau[0]))] = True
+        assert np.array_equal(mb[0, 0, b], want), b
