@@ -236,7 +236,9 @@ int score_impl(const void* Q, const void* K, const xattn_shape* shape, const Per
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* part = static_cast<float*>(ws);
   if ((rc = score_partials(Q, K, D, perm, part, st)) != XATTN_OK) return rc;
-  return cuda_status(launch_score_reduce(D, part, probs, st));
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(&ds)) != XATTN_OK) return rc;
+  return cuda_status(launch_score_reduce(D, part, probs, ds->status, st));
 }
 
 // Per-head thresholds from a host array; INVALID_ARG unless each is in (0, 1].
@@ -270,10 +272,13 @@ int score_select_impl(const void* Q, const void* K, const xattn_shape* shape, co
   PermArg perm;  // the antidiagonal
   std::memset(&perm, 0, sizeof(perm));
   for (int i = 0; i < D.S; ++i) perm.q[i] = static_cast<uint8_t>(D.S - 1 - i);
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(&ds)) != XATTN_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* part = static_cast<float*>(ws);
   if ((rc = score_partials(Q, K, D, perm, part, st)) != XATTN_OK) return rc;
-  return cuda_status(launch_score_select(D, part, probs, ta, mask, counts, idx, st));
+  return cuda_status(launch_score_select(D, part, probs, ta, mask, counts, idx, ds->status,
+                                         ds->num_sms, st));
 }
 
 // Fixed-budget selection (arguments already validated into `budget`).

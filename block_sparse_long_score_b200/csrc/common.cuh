@@ -78,7 +78,7 @@ cudaError_t launch_score_simt(const Dims& D, const float* Q, const float* K,
                               const PermArg& perm, float* part, cudaStream_t st);
 
 // partials -> block probabilities P [bh, NB, NB].
-cudaError_t launch_score_reduce(const Dims& D, const float* part, float* probs,
+cudaError_t launch_score_reduce(const Dims& D, const float* part, float* probs, int* status,
                                 cudaStream_t st);
 
 // Per-head thresholds: read from the device array `dev` when it is set (the
@@ -108,10 +108,33 @@ cudaError_t launch_select(const Dims& D, const float* probs, const TauArg& tau, 
                           int32_t* counts, int32_t* idx, int num_sms, cudaStream_t st);
 
 // partials -> P (optional) and find_blocks, fused (same outputs as
-// launch_score_reduce followed by launch_select).
+// launch_score_reduce followed by launch_select); num_sms sizes the grid of
+// the histogram search for rows the threshold filter leaves. `status` receives
+// time-outs of the kernel's bounded waits.
 cudaError_t launch_score_select(const Dims& D, const float* part, float* probs,
                                 const TauArg& tau, uint32_t* mask, int32_t* counts, int32_t* idx,
-                                cudaStream_t st);
+                                int* status, int num_sms, cudaStream_t st);
+
+// Where the histogram search finds the P row of a marked row: in P itself
+// ([rows][NB], layout 0), or written over the first partials of the row's
+// query block (layout 1: part + bh * part_head + part_row_offset(b * r)).
+struct RowSource {
+  const float* p;
+  int layout;
+  size_t part_head;
+  int r;
+};
+
+// find_blocks on every row of P read from `src` (the threshold filter, then
+// the histogram search on the rows it leaves).
+cudaError_t launch_select_rows(const Dims& D, const RowSource& src, const TauArg& tau,
+                               uint32_t* mask, int32_t* counts, int32_t* idx, int num_sms,
+                               cudaStream_t st);
+
+// The histogram search of find_blocks on the rows marked with count -1.
+cudaError_t launch_select_fallback(const Dims& D, const RowSource& src, const TauArg& tau,
+                                   uint32_t* mask, int32_t* counts, int32_t* idx, int num_sms,
+                                   cudaStream_t st);
 
 // One CTA whose bounded wait runs out (failure-detection self-test).
 cudaError_t launch_selftest_timeout(int* status, cudaStream_t st);

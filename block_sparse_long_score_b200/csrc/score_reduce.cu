@@ -36,8 +36,11 @@ __global__ void __launch_bounds__(kThreads)
 
 }  // namespace
 
-cudaError_t launch_score_reduce(const Dims& D, const float* part, float* probs,
-                                cudaStream_t st) {
+// Shapes the staged kernel of score_bulk.cu does not take (r outside 4..32, or
+// a workspace that is not 16-byte aligned): the two-pass reduce of
+// reduce_core.cuh straight from global memory.
+cudaError_t launch_score_reduce_wide(const Dims& D, const float* part, float* probs,
+                                     cudaStream_t st) {
   dim3 grid(D.NB, D.batch * D.hq);
   const size_t smem = ((D.r + 1) & ~1) * sizeof(float) + D.r * sizeof(size_t);
   score_reduce_kernel<<<grid, kThreads, smem, st>>>(part, probs, D.NB, D.r, D.R, D.causal);

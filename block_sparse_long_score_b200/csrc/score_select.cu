@@ -85,9 +85,11 @@ __global__ void __launch_bounds__(kThreads)
 
 }  // namespace
 
-cudaError_t launch_score_select(const Dims& D, const float* part, float* probs,
-                                const TauArg& tau, uint32_t* mask, int32_t* counts, int32_t* idx,
-                                cudaStream_t st) {
+// Shapes the staged kernel of score_bulk.cu does not take (r outside 4..32, or
+// a workspace that is not 16-byte aligned).
+cudaError_t launch_score_select_wide(const Dims& D, const float* part, float* probs,
+                                     const TauArg& tau, uint32_t* mask, int32_t* counts,
+                                     int32_t* idx, cudaStream_t st) {
   const int nb_stage = (D.NB + 3) & ~3;
   const size_t smem = sizeof(sel::WarpSmem) + sizeof(filt::WarpBuf) +
                       static_cast<size_t>(nb_stage) * 4 +

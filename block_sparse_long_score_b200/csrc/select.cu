@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(kBudgetWarps * 32)
 constexpr int kFiltWarps = 8;
 
 __global__ void __launch_bounds__(kFiltWarps * 32, 3)
-    select_filter_kernel(const float* __restrict__ probs, const TauArg tau, int NB, int hq,
+    select_filter_kernel(const RowSource src, const TauArg tau, int NB, int hq,
                          int causal, long long rows, uint32_t* __restrict__ mask,
                          int32_t* __restrict__ counts, int32_t* __restrict__ idx) {
   __shared__ filt::WarpBuf bufs[kFiltWarps];
@@ -180,7 +180,11 @@ __global__ void __launch_bounds__(kFiltWarps * 32, 3)
   const int h = static_cast<int>(bh % hq);
   const int n = causal ? b + 1 : NB;
   const double t = tau_of(tau, h);
-  const float* prow = probs + row * NB;
+  const float* prow =
+      src.layout == 0
+          ? src.p + row * NB
+          : src.p + static_cast<size_t>(bh) * src.part_head +
+                part_row_offset(b * src.r, src.r, NB, causal != 0);
 
   unsigned long long cut = 0;
   int ncand = 0;
@@ -207,7 +211,7 @@ __global__ void __launch_bounds__(kFiltWarps * 32, 3)
 
 // The histogram search of one row (select_core.cuh), with its keys staged in
 // the warp's shared memory.
-__device__ __forceinline__ void select_row_hist(const float* __restrict__ probs, const TauArg& tau,
+__device__ __forceinline__ void select_row_hist(const RowSource& src, const TauArg& tau,
                                                 int NB, int hq, int causal, long long row,
                                                 WarpSmem& W, uint32_t* keys, int lane,
                                                 uint32_t* __restrict__ mask,
@@ -217,8 +221,12 @@ __device__ __forceinline__ void select_row_hist(const float* __restrict__ probs,
   const int b = static_cast<int>(row % NB);
   const int h = static_cast<int>(bh % hq);
   const int n = causal ? b + 1 : NB;
-  const double t = tau_of(tau, h);  // valid: the fast kernel only leaves rows of valid tau
-  const float* prow = probs + row * NB;
+  const double t = tau_of(tau, h);  // valid: the filter only leaves rows of valid tau
+  const float* prow =
+      src.layout == 0
+          ? src.p + row * NB
+          : src.p + static_cast<size_t>(bh) * src.part_head +
+                part_row_offset(b * src.r, src.r, NB, causal != 0);
 
   double tot = 0.0;
   uint32_t kmax = 0;
@@ -255,7 +263,7 @@ __device__ __forceinline__ void select_row_hist(const float* __restrict__ probs,
 // Persistent: warp g of G owns rows g, g + G, g + 2G, ... and runs the
 // histogram search on those the fast kernel marked.
 __global__ void __launch_bounds__(kThreads)
-    select_fallback_kernel(const float* __restrict__ probs, const TauArg tau, int NB, int hq,
+    select_fallback_kernel(const RowSource src, const TauArg tau, int NB, int hq,
                            int causal, long long rows, int nb_stage, uint32_t* __restrict__ mask,
                            int32_t* __restrict__ counts, int32_t* __restrict__ idx) {
   extern __shared__ __align__(16) uint8_t smem[];
@@ -272,7 +280,7 @@ __global__ void __launch_bounds__(kThreads)
     while (todo) {
       const int q = __ffs(todo) - 1;
       todo &= todo - 1;
-      select_row_hist(probs, tau, NB, hq, causal, r0 + q * G, W, keys, lane, mask, counts, idx);
+      select_row_hist(src, tau, NB, hq, causal, r0 + q * G, W, keys, lane, mask, counts, idx);
     }
   }
 }
@@ -295,19 +303,33 @@ cudaError_t launch_select_budget(const Dims& D, const float* probs, const Budget
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const Dims& D, const float* probs, const TauArg& tau, uint32_t* mask,
-                          int32_t* counts, int32_t* idx, int num_sms, cudaStream_t st) {
+cudaError_t launch_select_rows(const Dims& D, const RowSource& src, const TauArg& tau,
+                               uint32_t* mask, int32_t* counts, int32_t* idx, int num_sms,
+                               cudaStream_t st) {
   const long long rows = static_cast<long long>(D.batch) * D.hq * D.NB;
   const long long filt_grid = (rows + kFiltWarps - 1) / kFiltWarps;
   select_filter_kernel<<<static_cast<unsigned>(filt_grid), kFiltWarps * 32, 0, st>>>(
-      probs, tau, D.NB, D.hq, D.causal, rows, mask, counts, idx);
-  cudaError_t e = cudaGetLastError();
+      src, tau, D.NB, D.hq, D.causal, rows, mask, counts, idx);
+  const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  return launch_select_fallback(D, src, tau, mask, counts, idx, num_sms, st);
+}
 
+cudaError_t launch_select(const Dims& D, const float* probs, const TauArg& tau, uint32_t* mask,
+                          int32_t* counts, int32_t* idx, int num_sms, cudaStream_t st) {
+  const RowSource src{probs, 0, 0, 0};
+  return launch_select_rows(D, src, tau, mask, counts, idx, num_sms, st);
+}
+
+cudaError_t launch_select_fallback(const Dims& D, const RowSource& src, const TauArg& tau,
+                                   uint32_t* mask, int32_t* counts, int32_t* idx, int num_sms,
+                                   cudaStream_t st) {
+  const long long rows = static_cast<long long>(D.batch) * D.hq * D.NB;
   const int nb_stage = (D.NB + 3) & ~3;
   const size_t smem = static_cast<size_t>(kWarps) * (sizeof(WarpSmem) + nb_stage * 4);
-  e = cudaFuncSetAttribute(select_fallback_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(select_fallback_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_fallback_kernel, kThreads,
@@ -317,7 +339,7 @@ cudaError_t launch_select(const Dims& D, const float* probs, const TauArg& tau, 
   const long long need = (rows + kWarps - 1) / kWarps;
   const long long grid = need < full ? need : full;
   select_fallback_kernel<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(
-      probs, tau, D.NB, D.hq, D.causal, rows, nb_stage, mask, counts, idx);
+      src, tau, D.NB, D.hq, D.causal, rows, nb_stage, mask, counts, idx);
   return cudaGetLastError();
 }
 
