@@ -41,12 +41,14 @@ WORKLOAD = "c2"   # the 128K Llama-shaped layer the metric is quoted on
 # the current kernels, for the workloads where a capture exists. The captures
 # ran the 8-query-head case of the same layer (bench.py --heads 8: 2 of the 8
 # KV groups, every query block); traffic grows with the number of heads, so the
-# figures are scaled by 32 / 8 to a full call. Summaries: profiles/.
+# figures are scaled by 32 / 8 to a full call. ncu flushes the caches before
+# every captured launch, so these are cold-cache figures. Summaries: profiles/.
 TRAFFIC_BYTES = {
-    # score_tc (CTA pairs) 390.05 MB read + 122.84 MB written; score_reduce 134.37 + 18.59 MB
-    ("c2", "score"): 4 * (390.05 + 122.84 + 134.37 + 18.59) * 1e6,
-    # attn_tc 864.53 MB read + 237.99 MB written (sched_kernel: 1.14 MB)
-    ("c2", "sparse_attn"): 4 * (864.53 + 237.99 + 1.14) * 1e6,
+    # xattn_score_select: score_tc 387.63 MB read + 120.76 MB written; score_bulk
+    # 134.40 + 5.10; select_filter 17.76 + 0; select_fallback 0.30 + 0
+    ("c2", "score_select"): 4 * (387.63 + 120.76 + 134.40 + 5.10 + 17.76 + 0.30) * 1e6,
+    # xattn_sparse_attn: attn_tc 863.92 MB read + 233.66 MB written; sched 1.14 MB
+    ("c2", "sparse_attn"): 4 * (863.92 + 233.66 + 1.14) * 1e6,
 }
 
 

@@ -262,7 +262,9 @@ __device__ __forceinline__ void select_row_hist(const RowSource& src, const TauA
 
 // Persistent: warp g of G owns rows g, g + G, g + 2G, ... and runs the
 // histogram search on those the fast kernel marked.
-__global__ void __launch_bounds__(kThreads)
+constexpr int kFbWarps = 1;
+
+__global__ void __launch_bounds__(kFbWarps * 32)
     select_fallback_kernel(const RowSource src, const TauArg tau, int NB, int hq,
                            int causal, long long rows, int nb_stage, uint32_t* __restrict__ mask,
                            int32_t* __restrict__ counts, int32_t* __restrict__ idx) {
@@ -272,8 +274,8 @@ __global__ void __launch_bounds__(kThreads)
   WarpSmem& W = *reinterpret_cast<WarpSmem*>(wbase);
   uint32_t* keys = reinterpret_cast<uint32_t*>(wbase + sizeof(WarpSmem));
 
-  const long long G = static_cast<long long>(gridDim.x) * kWarps;
-  const long long g = static_cast<long long>(blockIdx.x) * kWarps + warp;
+  const long long G = static_cast<long long>(gridDim.x) * kFbWarps;
+  const long long g = static_cast<long long>(blockIdx.x) * kFbWarps + warp;
   for (long long r0 = g; r0 < rows; r0 += 32 * G) {
     const long long r = r0 + lane * G;
     unsigned todo = __ballot_sync(0xffffffffu, r < rows && counts[r] < 0);
@@ -326,19 +328,15 @@ cudaError_t launch_select_fallback(const Dims& D, const RowSource& src, const Ta
                                    cudaStream_t st) {
   const long long rows = static_cast<long long>(D.batch) * D.hq * D.NB;
   const int nb_stage = (D.NB + 3) & ~3;
-  const size_t smem = static_cast<size_t>(kWarps) * (sizeof(WarpSmem) + nb_stage * 4);
-  cudaError_t e = cudaFuncSetAttribute(select_fallback_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
+  const size_t smem = static_cast<size_t>(kFbWarps) * (sizeof(WarpSmem) + nb_stage * 4);
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_fallback_kernel, kThreads,
-                                                    smem);
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_fallback_kernel,
+                                                                kFbWarps * 32, smem);
   if (e != cudaSuccess) return e;
   const long long full = static_cast<long long>(num_sms) * (per_sm > 0 ? per_sm : 1);
-  const long long need = (rows + kWarps - 1) / kWarps;
+  const long long need = (rows + kFbWarps - 1) / kFbWarps;
   const long long grid = need < full ? need : full;
-  select_fallback_kernel<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(
+  select_fallback_kernel<<<static_cast<unsigned>(grid), kFbWarps * 32, smem, st>>>(
       src, tau, D.NB, D.hq, D.causal, rows, nb_stage, mask, counts, idx);
   return cudaGetLastError();
 }
