@@ -195,6 +195,7 @@ int check_score_args(const void* Q, const void* K, const xattn_shape* shape, voi
   if (!Q || !K) return XATTN_ERR_INVALID_ARG;
   const size_t need = xattn_score_workspace_bytes(shape);
   if (!ws || ws_bytes < need) return XATTN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 3u) != 0) return XATTN_ERR_INVALID_ARG;  // fp32 partials
   if (D->dtype == XATTN_BF16 && (!aligned16(Q) || !aligned16(K))) return XATTN_ERR_INVALID_ARG;
   return XATTN_OK;
 }

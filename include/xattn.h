@@ -107,9 +107,10 @@ size_t xattn_score_workspace_bytes(const xattn_shape* shape);
  * Q: [batch, hq, L, d], K: [batch, hkv, L, d], both of type shape->dtype and
  *    16-byte aligned.
  * probs: out, fp32 [batch, hq, NB, NB], fully written.
- * ws / ws_bytes: workspace of at least xattn_score_workspace_bytes(shape).
- * Errors: INVALID_ARG (NULL pointer, bad shape), UNSUPPORTED (dtype limits,
- * NB > XATTN_MAX_BLOCKS), WORKSPACE, CUDA.
+ * ws / ws_bytes: workspace of at least xattn_score_workspace_bytes(shape),
+ *          4-byte aligned (every CUDA allocation is).
+ * Errors: INVALID_ARG (NULL pointer, bad shape, misaligned ws), UNSUPPORTED
+ * (dtype limits, NB > XATTN_MAX_BLOCKS), WORKSPACE, CUDA.
  */
 int xattn_score(const void* Q, const void* K, const xattn_shape* shape, float* probs,
                 void* ws, size_t ws_bytes, void* stream);
@@ -152,7 +153,8 @@ int xattn_select(const float* probs, const float* tau, const xattn_shape* shape,
  *        to xattn_score's output when given.
  * mask, counts, idx: out, as for xattn_select, and bit-identical to
  *        xattn_select run on xattn_score's P.
- * ws / ws_bytes: the scoring workspace (xattn_score_workspace_bytes).
+ * ws / ws_bytes: the scoring workspace (xattn_score_workspace_bytes), 4-byte
+ *          aligned.
  * Errors: as for xattn_score and xattn_select.
  */
 int xattn_score_select(const void* Q, const void* K, const xattn_shape* shape, const float* tau,

@@ -204,6 +204,18 @@ def test_prefill_host_checks(lib):
     assert f(FAKE, FAKE, FAKE, ctypes.byref(wide), good, FAKE, None, 0, FAKE, big, None) == -2
 
 
+def test_misaligned_score_workspace_rejected(lib):
+    """The scoring workspace holds fp32 partials: a workspace pointer that is
+    not 4-byte aligned is refused on the host (INVALID_ARG), by both scoring
+    calls, before any device work."""
+    s = X.make_shape(1, 4, 2, 1024, 128, 128, 8, True, "bf16")
+    need = X.xattn_score_workspace_bytes(s)
+    bad_ws = ctypes.c_void_p(0x10002)
+    assert lib.xattn_score(FAKE, FAKE, ctypes.byref(s), FAKE, bad_ws, need, None) == -1
+    assert lib.xattn_score_select(FAKE, FAKE, ctypes.byref(s), FAKE, None, FAKE, FAKE, FAKE,
+                                  bad_ws, need, None) == -1
+
+
 def test_ragged_length_accepted(lib):
     """L = 1000 (not a multiple of B = 128, a multiple of S = 8): 8 blocks,
     the last of 104 tokens. The host checks pass (the call then fails only on
