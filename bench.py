@@ -77,6 +77,18 @@ def bf16_peak_for_clocks(pk: dict, clk: dict) -> tuple:
     return pk["bf16_sustained"], f"{pk['source']} bf16 sustained ({seen} in the timed region)"
 
 
+def launches_per_step(r: int, two_call: bool) -> int:
+    """Kernels of this library one headline step launches (bf16 path), as the
+    library dispatches them: the scoring GEMM; for r = B/S in 4..32 the staged
+    reduce, then the selection filter and its histogram fallback (xattn_score_select
+    and xattn_score + xattn_select alike), for other r one fused reduce + select
+    kernel (xattn_score_select) or the two-pass reduce plus the two selection
+    kernels (three calls); then the schedule and the attention."""
+    if two_call or 4 <= r <= 32:
+        return 6
+    return 4
+
+
 def split_config(args, world: int, hq: int, hkv: int) -> dict:
     """How the ranks share the work: whole-layer replicas, or one layer cut
     into contiguous KV-head ranges (the config's hq/hkv are then this rank's)."""
@@ -566,7 +578,8 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     # headline step (the product path)
     if per["score_select"] >= per["sparse_attn"]:
         dom, dom_tflops = "score_select", ss_tflops
-        dom_kernel = "xattn_score_select (score_tc_kernel + score_select_kernel)"
+        dom_kernel = ("xattn_score_select (score_tc_kernel, score_bulk_kernel, "
+                      "select_filter_kernel, select_fallback_kernel)")
     else:
         dom, dom_tflops = "sparse_attn", attn_tflops
         dom_kernel = "xattn_sparse_attn (sched_kernel + attn_tc_kernel)"
@@ -632,7 +645,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
         # library kernels launched in the headline's timed region: score_tc +
         # score_select + sched + attn_tc a step (three calls: score_tc +
         # score_reduce + select_filter + select_fallback + sched + attn_tc)
-        "gpu_launches": (6 if args.two_call else 4) * args.steps,
+        "gpu_launches": launches_per_step(prob.B // prob.S, args.two_call) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
