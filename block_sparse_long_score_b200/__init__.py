@@ -9,7 +9,8 @@ sampling) and ``xattn_select_topk`` / ``xattn_select_topratio`` (fixed
 budgets). ``xattn_prefill_host`` runs the whole step on host tensors with the
 host<->device copies overlapped with the compute, and ``xattn_prefill_varlen``
 on a batch of sequences of different lengths; ``xattn_check_lists`` validates
-block lists made elsewhere before they reach the attention. The library loads on first
+block lists made elsewhere before they reach the attention; ``xattn_score_partials``
+runs the scoring GEMM alone. The library loads on first
 use and the calls raise if it is missing.
 """
 from .xattn import (  # noqa: F401
@@ -19,6 +20,6 @@ from .xattn import (  # noqa: F401
     xattn_select_topk, xattn_select_topratio, antidiagonal_perm, diagonal_perm,
     xattn_score_select, xattn_selftest_timeout, xattn_prefill_host,
     xattn_prefill_host_workspace_bytes, xattn_prefill_varlen,
-    xattn_prefill_varlen_workspace_bytes, xattn_check_lists,
+    xattn_prefill_varlen_workspace_bytes, xattn_check_lists, xattn_score_partials,
 )
 from .pipeline import prefill_attention, prefill_buffers  # noqa: F401

@@ -308,6 +308,19 @@ int xattn_score(const void* Q, const void* K, const xattn_shape* shape, float* p
   return score_impl(Q, K, shape, perm, probs, ws, ws_bytes, stream);
 }
 
+int xattn_score_partials(const void* Q, const void* K, const xattn_shape* shape, void* ws,
+                         size_t ws_bytes, void* stream) {
+  Dims D;
+  int rc = check_score_args(Q, K, shape, ws, ws_bytes, &D);
+  if (rc != XATTN_OK) return rc;
+  if (D.S > 256) return XATTN_ERR_UNSUPPORTED;  // S divides B <= 256 for every valid shape
+  PermArg perm;  // the antidiagonal
+  std::memset(&perm, 0, sizeof(perm));
+  for (int i = 0; i < D.S; ++i) perm.q[i] = static_cast<uint8_t>(D.S - 1 - i);
+  return score_partials(Q, K, D, perm, static_cast<float*>(ws),
+                        static_cast<cudaStream_t>(stream));
+}
+
 int xattn_score_pattern(const void* Q, const void* K, const xattn_shape* shape,
                         const int32_t* perm, float* probs, void* ws, size_t ws_bytes,
                         void* stream) {

@@ -24,6 +24,7 @@ __all__ = [
     "antidiagonal_perm", "diagonal_perm", "xattn_score_select", "xattn_selftest_timeout",
     "xattn_prefill_host_workspace_bytes", "xattn_prefill_host",
     "xattn_prefill_varlen_workspace_bytes", "xattn_prefill_varlen", "xattn_check_lists",
+    "xattn_score_partials",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -37,6 +38,7 @@ EXPORTED_SYMBOLS = (
     "xattn_select_topk", "xattn_select_topratio", "xattn_score_select",
     "xattn_selftest_timeout", "xattn_prefill_host_workspace_bytes", "xattn_prefill_host",
     "xattn_prefill_varlen_workspace_bytes", "xattn_prefill_varlen", "xattn_check_lists",
+    "xattn_score_partials",
 )
 # batch * hq * NB limit of xattn_sparse_attn_noalloc (XATTN_NOALLOC_MAX_UNITS)
 NOALLOC_MAX_UNITS = 1 << 18
@@ -75,6 +77,8 @@ def _lib() -> ctypes.CDLL:
         lib.xattn_attn_workspace_bytes.argtypes = [sp]
         lib.xattn_attn_workspace_bytes.restype = sz
         lib.xattn_score.argtypes = [vp, vp, sp, vp, vp, sz, vp]
+        lib.xattn_score_partials.argtypes = [vp, vp, sp, vp, sz, vp]
+        lib.xattn_score_partials.restype = i32
         lib.xattn_score.restype = i32
         lib.xattn_select.argtypes = [vp, vp, sp, vp, vp, vp, vp]
         lib.xattn_select.restype = i32
@@ -232,6 +236,29 @@ def xattn_score(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal: bool,
     _same_device(Q, K, probs, workspace)
     with torch.cuda.device(Q.device):
         return _score_call(Q, K, S, shape, probs, workspace, perm)
+
+
+def xattn_score_partials(Q: torch.Tensor, K: torch.Tensor, B: int, S: int, causal: bool,
+                         workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The scoring GEMM alone: the per-key-block partial log2-sum-exp sums of
+    every reshaped query row, written to (and returned as) the uint8 scoring
+    workspace; the sums are its first fp32 entries, laid out as the header
+    states."""
+    _check(Q, "Q")
+    _check(K, "K", Q.dtype)
+    shape = _shape_of(Q, K, B, S, causal)
+    need = xattn_score_workspace_bytes(shape)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
+    _check(workspace, "workspace")
+    _same_device(Q, K, workspace)
+    with torch.cuda.device(Q.device):
+        rc = _lib().xattn_score_partials(Q.data_ptr(), K.data_ptr(), ctypes.byref(shape),
+                                         workspace.data_ptr(),
+                                         workspace.numel() * workspace.element_size(),
+                                         _stream(Q.device))
+    _raise("xattn_score_partials", rc)
+    return workspace
 
 
 def _score_call(Q, K, S, shape, probs, workspace, perm):

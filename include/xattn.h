@@ -44,6 +44,7 @@
  * The remaining calls have no counterpart in the paper; each is documented
  * where it is declared:
  *   xattn_score_select         scoring and find_blocks in one call (P kept on chip)
+ *   xattn_score_partials       the scoring GEMM alone (its partial sums, no P)
  *   xattn_sparse_attn_noalloc  the attention without a workspace
  *   xattn_check_lists          validation of block lists made by the caller
  *   xattn_prefill_host         the whole step on HOST buffers (the one call
@@ -180,6 +181,31 @@ int xattn_score_select(const void* Q, const void* K, const xattn_shape* shape, c
 int xattn_score_pattern(const void* Q, const void* K, const xattn_shape* shape,
                         const int32_t* perm, float* probs, void* ws, size_t ws_bytes,
                         void* stream);
+
+/*
+ * The first stage of xattn_score alone: the strided antidiagonal product
+ * (§2.1, Algorithm 1's Q_r K_r^T with the 1/sqrt(d*S) scale and the causal
+ * mask), reduced within each key block and written to the workspace. It is
+ * the tensor-core GEMM of the path by itself, for timing it on its own, and
+ * for callers that reduce the sums themselves.
+ *
+ * For each (batch, query head) bh, reshaped query row rho (0 <= rho < L/S) and
+ * allowed key block j (j <= rho / r when causal, all NB otherwise; r = B/S):
+ *   L[bh, rho, j] = log2 sum over the visible reshaped columns c of block j of
+ *                   2^(x[rho, c] * log2(e)),  x = Q_r K_r^T / sqrt(d*S)
+ * (fp32; a column c of block j is visible when c < L/S and, causal, c <= rho).
+ * Layout in ws (fp32): head bh starts at bh * H floats, H = r*NB*(NB+1)/2
+ * (causal) or (L/S)*NB; within a head, the row of rho starts at
+ * r*b*(b+1)/2 + t*(b+1) (causal, b = rho / r, t = rho % r) or rho*NB, and
+ * holds the row's allowed blocks j = 0, 1, ... in order. P follows as
+ * P[b, j] = (1/r_b) sum over the block's rows rho of 2^(L[rho, j] - LSE[rho]),
+ * LSE[rho] = log2 sum_j 2^L[rho, j].
+ *
+ * ws / ws_bytes: as for xattn_score (the sums occupy its first bytes).
+ * Errors: as for xattn_score.
+ */
+int xattn_score_partials(const void* Q, const void* K, const xattn_shape* shape, void* ws,
+                         size_t ws_bytes, void* stream);
 
 /*
  * Fixed-budget selection, the Top-K and Top-Ratio strategies of the

@@ -214,6 +214,20 @@ def test_misaligned_score_workspace_rejected(lib):
     assert lib.xattn_score(FAKE, FAKE, ctypes.byref(s), FAKE, bad_ws, need, None) == -1
     assert lib.xattn_score_select(FAKE, FAKE, ctypes.byref(s), FAKE, None, FAKE, FAKE, FAKE,
                                   bad_ws, need, None) == -1
+    assert lib.xattn_score_partials(FAKE, FAKE, ctypes.byref(s), bad_ws, need, None) == -1
+
+
+def test_score_partials_host_checks(lib):
+    """xattn_score_partials applies xattn_score's host checks: NULL inputs are
+    INVALID_ARG, a missing or short workspace is WORKSPACE, all before any
+    device work."""
+    s = X.make_shape(1, 4, 2, 1024, 128, 128, 8, True, "bf16")
+    need = X.xattn_score_workspace_bytes(s)
+    assert lib.xattn_score_partials(None, FAKE, ctypes.byref(s), FAKE, need, None) == -1
+    assert lib.xattn_score_partials(FAKE, None, ctypes.byref(s), FAKE, need, None) == -1
+    assert lib.xattn_score_partials(FAKE, FAKE, ctypes.byref(s), None, need, None) == -4
+    assert lib.xattn_score_partials(FAKE, FAKE, ctypes.byref(s), FAKE, need - 1, None) == -4
+    assert lib.xattn_score_partials(FAKE, FAKE, None, FAKE, need, None) == -1
 
 
 def test_ragged_length_accepted(lib):

@@ -74,6 +74,7 @@ def test_every_entry_point_applies_the_same_rules(lib, shp):
     assert X.xattn_prefill_host_workspace_bytes(s, 0) == 0
     calls = [
         lib.xattn_score(FAKE, FAKE, sref, FAKE, FAKE, 1 << 40, None),
+        lib.xattn_score_partials(FAKE, FAKE, sref, FAKE, 1 << 40, None),
         lib.xattn_score_select(FAKE, FAKE, sref, tau, None, FAKE, FAKE, FAKE, FAKE, 1 << 40,
                                None),
         lib.xattn_select(FAKE, tau, sref, FAKE, FAKE, FAKE, None),
