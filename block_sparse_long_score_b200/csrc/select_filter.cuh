@@ -13,10 +13,11 @@
 // the definition's walk up to the cut. The warp finds the row maximum m, then
 // tries theta = m * 2^-6, 2^-12, 2^-18 until the candidates' fp32 sum reaches
 // tau (within rounding), gathers the candidates in index order (at most
-// kCand of them) into shared memory, sorts them across the warp with a bitonic
-// network and walks them. A walk that covers every non-zero block without
-// reaching tau takes the whole row. Rows that need more than kCand candidates
-// (flat rows) are left to the histogram search (select_core.cuh).
+// kCand = 256 of them) into shared memory, sorts them across the warp with a
+// bitonic network (one to eight keys a lane) and walks them. A walk that
+// covers every non-zero block without reaching tau takes the whole row. Rows
+// that need more than kCand candidates (flat rows) are left to the histogram
+// search (select_core.cuh).
 //
 // The work per element is a handful of instructions (maximum, threshold sum,
 // ballot compaction); the sort, the walk and the emit depend on the number of
@@ -30,7 +31,7 @@
 namespace xattn {
 namespace filt {
 
-constexpr int kCand = 64;       // candidates a warp sorts (two per lane)
+constexpr int kCand = 256;      // candidates a warp sorts (up to eight per lane)
 constexpr int kMaxWords = XATTN_MAX_BLOCKS / 32;
 constexpr int kRegU = 32;       // row elements a lane holds in registers (n <= 1024)
 
@@ -86,43 +87,95 @@ struct MemRow {
   }
 };
 
-// Bitonic sort, descending, of one key a lane (32 keys).
-__device__ __forceinline__ unsigned long long sort32_desc(unsigned long long x, int lane) {
+// Bitonic sort, descending, of 32 * KPL keys held KPL a lane: k[q] is
+// position lane + 32 q. Partners 32 or more positions apart sit in the same
+// lane; closer ones are exchanged with warp shuffles.
+template <int KPL>
+__device__ __forceinline__ void sort_desc(unsigned long long (&k)[KPL], int lane) {
+  constexpr int N = 32 * KPL;
 #pragma unroll
-  for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      const unsigned long long o = __shfl_xor_sync(0xffffffffu, x, stride);
-      const bool take_max = ((lane & size) == 0) == ((lane & stride) == 0);
-      x = take_max ? (o > x ? o : x) : (o < x ? o : x);
-    }
-  }
-  return x;
-}
-
-// Bitonic sort, descending, of 64 keys held two a lane: a at position lane,
-// b at position lane + 32.
-__device__ __forceinline__ void sort64_desc(unsigned long long& a, unsigned long long& b,
-                                            int lane) {
-#pragma unroll
-  for (int size = 2; size <= 64; size <<= 1) {
+  for (int size = 2; size <= N; size <<= 1) {
 #pragma unroll
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      if (stride == 32) {  // partners sit in the same lane (only for size 64: descending)
-        const unsigned long long hi = a > b ? a : b, lo = a > b ? b : a;
-        a = hi;
-        b = lo;
+      if (stride >= 32) {
+        const int qs = stride / 32;
+#pragma unroll
+        for (int q = 0; q < KPL; ++q) {
+          if ((q & qs) != 0) continue;
+          // positions p (this entry) and p + stride (entry q | qs)
+          const bool up = ((lane + 32 * q) & size) == 0;  // descending run
+          const unsigned long long x = k[q], y = k[q | qs];
+          const unsigned long long hi = x > y ? x : y, lo = x > y ? y : x;
+          k[q] = up ? hi : lo;
+          k[q | qs] = up ? lo : hi;
+        }
       } else {
-        const unsigned long long oa = __shfl_xor_sync(0xffffffffu, a, stride);
-        const unsigned long long ob = __shfl_xor_sync(0xffffffffu, b, stride);
         const bool lower = (lane & stride) == 0;
-        const bool up_a = (lane & size) == 0;          // position lane
-        const bool up_b = ((lane + 32) & size) == 0;   // position lane + 32
-        a = (up_a == lower) ? (oa > a ? oa : a) : (oa < a ? oa : a);
-        b = (up_b == lower) ? (ob > b ? ob : b) : (ob < b ? ob : b);
+#pragma unroll
+        for (int q = 0; q < KPL; ++q) {
+          const unsigned long long o = __shfl_xor_sync(0xffffffffu, k[q], stride);
+          const bool up = ((lane + 32 * q) & size) == 0;
+          k[q] = (up == lower) ? (o > k[q] ? o : k[q]) : (o < k[q] ? o : k[q]);
+        }
       }
     }
   }
+}
+
+// Loads the c candidates (in index order) KPL a lane, sorts them descending
+// and finds where the ranked fp64 sum reaches t. True (and the cut key) if it
+// does.
+//
+// The definition adds one probability after another in fp64. With exact_sums
+// the candidates all lie within 19 binades below the row maximum (theta is at
+// least m * 2^-18), so each is a multiple of the smallest one's ulp and any
+// sum of at most 256 of them needs at most 18 + 24 + 8 = 50 significant bits:
+// every partial sum is exact in fp64, whatever the order of the additions. A
+// warp prefix scan then gives the very sums of the one-by-one walk, and the
+// cut is the first position where the scan reaches t. Otherwise (theta is the
+// smallest non-zero pattern) the walk adds one candidate after another.
+template <int KPL>
+__device__ __forceinline__ bool sort_walk(const WarpBuf& W, int c, double t, bool exact_sums,
+                                          int lane, unsigned long long* cut) {
+  unsigned long long k[KPL];
+#pragma unroll
+  for (int q = 0; q < KPL; ++q) k[q] = lane + 32 * q < c ? W.cand[lane + 32 * q] : 0ull;
+  sort_desc<KPL>(k, lane);
+  if (exact_sums) {
+    double carry = 0.0;  // sum of the positions before this group of 32
+#pragma unroll
+    for (int q = 0; q < KPL; ++q) {
+      if (32 * q >= c) break;  // warp-uniform
+      double incl = static_cast<double>(key_value(k[q]));  // 0 past c (key 0)
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, lane + 32 * q < c && carry + incl >= t);
+      if (hit) {
+        *cut = __shfl_sync(0xffffffffu, k[q], __ffs(hit) - 1);
+        return true;
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    return false;
+  }
+  double acc = 0.0;
+#pragma unroll
+  for (int q = 0; q < KPL; ++q) {
+    if (32 * q >= c) break;  // warp-uniform
+    const int m = min(32, c - 32 * q);
+    for (int ii = 0; ii < m; ++ii) {
+      const unsigned long long key = __shfl_sync(0xffffffffu, k[q], ii);
+      acc += static_cast<double>(key_value(key));
+      if (acc >= t) {
+        *cut = key;
+        return true;
+      }
+    }
+  }
+  return false;
 }
 
 // Outcome of the filter for one row.
@@ -174,23 +227,15 @@ __device__ __forceinline__ Outcome filter_cut(const Row& row, int n, double t, i
       base += __popc(b);
     });
     __syncwarp();
-    unsigned long long a = lane < c ? W.cand[lane] : 0ull;
-    unsigned long long b = lane + 32 < c ? W.cand[lane + 32] : 0ull;
-    if (c <= 32) {
-      a = sort32_desc(a, lane);
-    } else {
-      sort64_desc(a, b, lane);
-    }
     // the definition's walk: ranked order, one fp64 addition after another
-    double acc = 0.0;
-    for (int i = 0; i < c; ++i) {
-      const unsigned long long key = __shfl_sync(0xffffffffu, i < 32 ? a : b, i & 31);
-      acc += static_cast<double>(key_value(key));
-      if (acc >= t) {
-        *cut = key;
-        *ncand = c;
-        return kCut;
-      }
+    const bool ex = !all_nonzero;
+    const bool reached = c <= 32   ? sort_walk<1>(W, c, t, ex, lane, cut)
+                         : c <= 64  ? sort_walk<2>(W, c, t, ex, lane, cut)
+                         : c <= 128 ? sort_walk<4>(W, c, t, ex, lane, cut)
+                                    : sort_walk<8>(W, c, t, ex, lane, cut);
+    if (reached) {
+      *ncand = c;
+      return kCut;
     }
     if (all_nonzero) return kTakeAll;  // the whole row sums to less than t
     __syncwarp();  // the next attempt overwrites the candidates
