@@ -122,3 +122,28 @@ def test_cut_below_the_first_thresholds_and_zero_rows():
                 row[:] = 0.0
             P[0, h, b, :n] = row
     _check(P, [0.5 + 0.5 * 2.0 ** -9 * 7.5, 0.5 + 0.5 * 2.0 ** -15 * 12.5, 0.6, 0.9], True)
+
+
+@pytest.mark.parametrize("k", [32, 33, 64, 65, 128, 129, 200, 256, 257, 400])
+def test_candidate_counts_around_the_filter_sizes(k):
+    """Rows whose threshold that first reaches tau holds exactly k candidates:
+    one to eight keys a lane in the filter's sort (k <= 256), the histogram
+    search above that. The candidates take a few distinct values within a
+    factor of 8, and many tie, so both the ranked order and the exact prefix
+    scan of the walk are exercised; tau falls between and exactly on ranked
+    sums."""
+    NB = 512
+    rng = np.random.default_rng(k)
+    P = np.zeros((1, 3, NB, NB))
+    for h in range(3):
+        for b in range(NB):
+            row = np.full(NB, 2.0 ** -30)
+            pos = rng.choice(NB, size=k, replace=False)
+            row[pos] = rng.choice([1.0, 1.0, 0.5, 0.25, 0.125], size=k)
+            row /= row.sum()
+            P[0, h, b] = row
+    P32 = P.astype(np.float32).astype(np.float64)
+    # head 2: tau exactly equal to a ranked fp64 partial sum (cut on the boundary)
+    ranked = np.sort(P32[0, 2, 0])[::-1]
+    tau2 = float(np.float32(np.cumsum(ranked)[k // 2]))
+    _check(P, [0.5, 0.9, tau2], False)
