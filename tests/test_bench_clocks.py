@@ -102,3 +102,17 @@ def test_cpu_baseline_scales_setup_and_units_apart(monkeypatch):
     assert cb["kind"] == "oracle" and cb["unit"] == "ms/layer" and cb["extrapolated"]
     assert cb["value"] > 0 and cb["measured_s"] > 0
     assert "query heads [0, 3] of 4 x 4 of 8 query blocks" in cb["sample"]
+
+
+def test_launch_count_follows_the_dispatch():
+    """gpu_launches per headline step: the scoring GEMM, then for r = B/S in
+    4..32 the staged reduce, the selection filter and its fallback (the
+    product path and the three calls alike), for other r the one-kernel fused
+    reduce + select (product path) or the two-pass reduce and both selection
+    kernels (three calls); then the schedule and the attention."""
+    import bench
+    assert bench.launches_per_step(8, False) == 6    # c2: S = 16, r = 8
+    assert bench.launches_per_step(32, False) == 6   # S = 4
+    assert bench.launches_per_step(4, True) == 6
+    assert bench.launches_per_step(2, False) == 4    # S = 64: fused wide kernel
+    assert bench.launches_per_step(1, True) == 6
