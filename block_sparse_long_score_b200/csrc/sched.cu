@@ -25,8 +25,8 @@ namespace {
 
 constexpr int kThreads = 1024;
 
-// Effective block count and mask flag (bit 48) of the 8 consecutive units
-// u .. u + 7: causal lists drop trailing blocks above the diagonal.
+// Effective block count and mask flag (bit 48) of units u, u + kThreads, ...
+// (8 of them): causal lists drop trailing blocks above the diagonal.
 __device__ __forceinline__ void unit_info8(const int32_t* __restrict__ counts,
                                            const int32_t* __restrict__ idx, int u, int units,
                                            int NB, int causal, int ragged, int (&n)[8],
@@ -34,7 +34,7 @@ __device__ __forceinline__ void unit_info8(const int32_t* __restrict__ counts,
   int c[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
-    const int uu = u + q;
+    const int uu = u + q * kThreads;
     const int v = uu < units ? counts[uu] : 0;
     c[q] = v < 0 ? 0 : (v > NB ? NB : v);
   }
@@ -42,12 +42,12 @@ __device__ __forceinline__ void unit_info8(const int32_t* __restrict__ counts,
     int last[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      const int uu = u + q;
+      const int uu = u + q * kThreads;
       last[q] = (uu < units && c[q] > 0) ? idx[static_cast<size_t>(uu) * NB + c[q] - 1] : -1;
     }
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      const int uu = u + q;
+      const int uu = u + q * kThreads;
       const int qb = uu % NB;
       if (uu < units && last[q] > qb) {  // rare: trailing blocks above the diagonal
         const int32_t* list = idx + static_cast<size_t>(uu) * NB;
@@ -61,7 +61,7 @@ __device__ __forceinline__ void unit_info8(const int32_t* __restrict__ counts,
     // can only be a list's last entry
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      const int uu = u + q;
+      const int uu = u + q * kThreads;
       diag[q] = uu < units && c[q] > 0 && idx[static_cast<size_t>(uu) * NB + c[q] - 1] == NB - 1;
     }
   } else {
@@ -89,33 +89,17 @@ __global__ void __launch_bounds__(kThreads)
   const int ngrouped = groups > 1 ? groups * (NB + 1) : 0;
   for (int i = threadIdx.x; i < NB + 1 + ngrouped; i += kThreads) bins[i] = 0;
   __syncthreads();
-  // 8 consecutive units per thread per batch (neighbouring query blocks of one
-  // head, whose lists are often equally long): their load chains overlap, and a
-  // run of equal bins costs one shared-memory atomic
+  // 8 units per thread per batch: their load chains overlap
   for (int u0 = 0; u0 < units; u0 += 8 * kThreads) {
-    const int ub = u0 + 8 * threadIdx.x;
     int n[8];
     bool diag[8];
-    unit_info8(counts, idx, ub, units, NB, causal, ragged, n, diag);
-    int gb[8];  // grouped bin (or the plain one)
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      gb[q] = ngrouped ? ((ub + q) / units_per_group) * (NB + 1) + NB - n[q] : NB - n[q];
-    int run_p = 0, run_g = 0;
+    unit_info8(counts, idx, u0 + threadIdx.x, units, NB, causal, ragged, n, diag);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      if (ub + q >= units) break;
-      ++run_p;
-      ++run_g;
-      const bool more = q + 1 < 8 && ub + q + 1 < units;
-      if (!(more && n[(q + 1) & 7] == n[q])) {
-        atomicAdd(&plain[NB - n[q]], run_p);
-        run_p = 0;
-      }
-      if (ngrouped && !(more && gb[(q + 1) & 7] == gb[q])) {
-        atomicAdd(&grouped[gb[q]], run_g);
-        run_g = 0;
-      }
+      const int u = u0 + threadIdx.x + q * kThreads;
+      if (u >= units) continue;
+      atomicAdd(&plain[NB - n[q]], 1);
+      if (ngrouped) atomicAdd(&grouped[(u / units_per_group) * (NB + 1) + NB - n[q]], 1);
     }
   }
   __syncthreads();
@@ -169,28 +153,15 @@ __global__ void __launch_bounds__(kThreads)
   }
   __syncthreads();
   for (int u0 = 0; u0 < units; u0 += 8 * kThreads) {
-    const int ub = u0 + 8 * threadIdx.x;
     int n[8];
     bool diag[8];
-    unit_info8(counts, idx, ub, units, NB, causal, ragged, n, diag);
-    int bin[8], rl[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      bin[q] = by_group ? ((ub + q) / units_per_group) * (NB + 1) + NB - n[q] : NB - n[q];
-    // rl[q]: length of the run of equal bins that starts at q
-#pragma unroll
-    for (int q = 7; q >= 0; --q) {
-      const bool more = q + 1 < 8 && ub + q + 1 < units;
-      rl[q] = (more && bin[(q + 1) & 7] == bin[q]) ? rl[(q + 1) & 7] + 1 : 1;
-    }
-    int next = 0;  // position of the next unit of the current run
+    unit_info8(counts, idx, u0 + threadIdx.x, units, NB, causal, ragged, n, diag);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      const int u = ub + q;
-      if (u >= units) break;
-      const bool start = q == 0 || bin[(q + 7) & 7] != bin[q];
-      if (start) next = atomicAdd(&hist[bin[q]], rl[q]);
-      int pos = next++;
+      const int u = u0 + threadIdx.x + q * kThreads;
+      if (u >= units) continue;
+      const int bin = by_group ? (u / units_per_group) * (NB + 1) + NB - n[q] : NB - n[q];
+      int pos = atomicAdd(&hist[bin], 1);
       // the attention CTAs deal the order out in rounds of `ctas` units (CTA
       // i takes entries i, i + ctas, ...); every other round runs backwards,
       // so the CTA that gets a round's longest unit gets the next round's
