@@ -81,12 +81,12 @@ def bf16_peak_for_clocks(pk: dict, clk: dict) -> tuple:
 
 def launches_per_step(r: int, two_call: bool) -> int:
     """Kernels of this library one headline step launches (bf16 path), as the
-    library dispatches them: the scoring GEMM; for r = B/S in 4..32 the staged
+    library dispatches them: the scoring GEMM; for r = B/S in 1..32 the staged
     reduce, then the selection filter and its histogram fallback (xattn_score_select
     and xattn_score + xattn_select alike), for other r one fused reduce + select
     kernel (xattn_score_select) or the two-pass reduce plus the two selection
     kernels (three calls); then the schedule and the attention."""
-    if two_call or 4 <= r <= 32:
+    if two_call or 1 <= r <= 32:
         return 6
     return 4
 

@@ -41,7 +41,7 @@ namespace {
 
 constexpr int kThreads = 128;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMinR = 4, kMaxR = 32;        // r this kernel takes (bulk copies stay aligned)
+constexpr int kMinR = 1, kMaxR = 32;        // r this kernel takes
 constexpr int kStageCap = 32 * 1024 / 4;    // floats of the staging buffer at most
 
 __global__ void __launch_bounds__(kThreads)

@@ -36,8 +36,9 @@ __global__ void __launch_bounds__(kThreads)
 
 }  // namespace
 
-// Shapes the staged kernel of score_bulk.cu does not take (r outside 4..32, or
-// a workspace that is not 16-byte aligned): the two-pass reduce of
+// Shapes the staged kernel of score_bulk.cu does not take (r above 32, i.e.
+// strides 1 and 2 at B = 128, or a workspace that is not 16-byte aligned): the
+// two-pass reduce of
 // reduce_core.cuh straight from global memory.
 cudaError_t launch_score_reduce_wide(const Dims& D, const float* part, float* probs,
                                      cudaStream_t st) {

@@ -85,8 +85,8 @@ __global__ void __launch_bounds__(kThreads)
 
 }  // namespace
 
-// Shapes the staged kernel of score_bulk.cu does not take (r outside 4..32, or
-// a workspace that is not 16-byte aligned).
+// Shapes the staged kernel of score_bulk.cu does not take (r above 32, i.e.
+// strides 1 and 2 at B = 128, or a workspace that is not 16-byte aligned).
 cudaError_t launch_score_select_wide(const Dims& D, const float* part, float* probs,
                                      const TauArg& tau, uint32_t* mask, int32_t* counts,
                                      int32_t* idx, cudaStream_t st) {

@@ -106,7 +106,7 @@ def test_cpu_baseline_scales_setup_and_units_apart(monkeypatch):
 
 def test_launch_count_follows_the_dispatch():
     """gpu_launches per headline step: the scoring GEMM, then for r = B/S in
-    4..32 the staged reduce, the selection filter and its fallback (the
+    1..32 the staged reduce, the selection filter and its fallback (the
     product path and the three calls alike), for other r the one-kernel fused
     reduce + select (product path) or the two-pass reduce and both selection
     kernels (three calls); then the schedule and the attention."""
@@ -114,5 +114,6 @@ def test_launch_count_follows_the_dispatch():
     assert bench.launches_per_step(8, False) == 6    # c2: S = 16, r = 8
     assert bench.launches_per_step(32, False) == 6   # S = 4
     assert bench.launches_per_step(4, True) == 6
-    assert bench.launches_per_step(2, False) == 4    # S = 64: fused wide kernel
-    assert bench.launches_per_step(1, True) == 6
+    assert bench.launches_per_step(2, False) == 6    # S = 64
+    assert bench.launches_per_step(64, False) == 4   # S = 2: fused wide kernel
+    assert bench.launches_per_step(128, True) == 6
