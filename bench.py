@@ -677,9 +677,11 @@ def baseline_heads(hq: int) -> list:
 
 def run_reference(args, rank: int, world: int) -> None:
     """The oracle on the host cores: a bounded sample of the same workload per
-    step, in the same unit. Step i samples query head (i * (hq/4 + 1)) mod hq
-    on 128 evenly spread query blocks, so the steps walk over every head; the
-    value is the mean of the steps' whole-layer estimates."""
+    step, in the same unit. Step i samples one of the in-bench CPU baseline's
+    query heads (baseline_heads: every KV group, and on the 128K layer every
+    tau value) in turn, on 128 evenly spread query blocks; the value is the
+    mean of the steps' whole-layer estimates. Both legs therefore time the
+    same heads."""
     if rank != 0:
         return
     from block_sparse_long_score_b200.synth import make_problem
@@ -689,8 +691,9 @@ def run_reference(args, rank: int, world: int) -> None:
     vals, measured, heads = [], 0.0, []
     cb = None
     steps = max(1, args.steps)
+    pool = baseline_heads(prob.hq)
     for i in range(steps):
-        h = (i * (prob.hq // 4 + 1)) % prob.hq
+        h = pool[i % len(pool)]
         heads.append(h)
         cb = oracle_sample(prob, [h], n_blocks=128)
         vals.append(cb["value"])
@@ -698,8 +701,8 @@ def run_reference(args, rank: int, world: int) -> None:
     v = float(np.mean(vals))
     cb["value"] = v
     cb["measured_s"] = measured
-    cb["sample"] = (f"{steps} steps, step i = query head (i * {prob.hq // 4 + 1}) mod {prob.hq} "
-                    f"(heads {sorted(set(heads))}) x 128 evenly spread query blocks; "
+    cb["sample"] = (f"{steps} steps, step i = query head {pool}[i mod {len(pool)}] of "
+                    f"{prob.hq} (the in-bench baseline's heads) x 128 evenly spread query blocks; "
                     f"{measured:.1f} s of oracle work measured in all; each step's time "
                     f"scaled to the whole layer (per-head set-up x heads, per-block work x "
                     f"units) and averaged. Inputs converted to float64 before timing")
